@@ -1,0 +1,130 @@
+"""fp64 CPU oracle for non-causal multi-head attention (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports it, and it imports nothing from them: the
+two share no code.  The arithmetic lives in ``attention_oracle.c`` (plain C,
+double precision, OpenMP over rows); this module only compiles it with gcc and
+marshals numpy arrays through ctypes.
+
+What it computes, per batch b and head h, on token-major ``[B, N, H, D]``
+inputs (hf2q ``src/inference/vision/vit_gpu.rs``, doc of ``vit_attention_gpu``
+and ``vit_attention_scores_gpu``; inferencelayer ``src/vision_gpu.rs``,
+``vis_attn_coop_src`` doc, "Shape")::
+
+    s_ij  = scale * Q[i] . K[j]
+    p_ij  = softmax_j(s_ij)          (row maximum subtracted first)
+    O[i]  = sum_j p_ij V[j]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attention_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+BF16, F16, F64 = 0, 1, 2
+MODE_TWO_PASS, MODE_LSE, MODE_BRUTE = 0, 1, 2
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/liboracle.so`` (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+               "-ffp-contract=off", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        p, i64, dbl, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_double, ctypes.c_int
+        lib.oracle_attention.argtypes = [p, p, p, i64, i64, i64, i64, dbl, i32, i32, p]
+        lib.oracle_attention_rows.argtypes = [p, p, p, i64, i64, i64, i64, dbl, i32, i32, p, i64, p]
+        lib.oracle_attention_probs.argtypes = [p, p, i64, i64, i64, i64, dbl, i32, i64, i64, p]
+        lib.oracle_widen.argtypes = [p, i64, i32, p]
+        for f in (lib.oracle_attention, lib.oracle_attention_rows, lib.oracle_attention_probs,
+                  lib.oracle_widen, lib.oracle_num_threads):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _as_input(x: np.ndarray, dtype: int) -> np.ndarray:
+    want = np.float64 if dtype == F64 else np.uint16
+    x = np.ascontiguousarray(x)
+    if x.dtype != want:
+        raise TypeError(f"oracle input must be {want.__name__} for dtype code {dtype}, got {x.dtype}")
+    return x
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def attention(q, k, v, scale: float, dtype: int, mode: int = MODE_TWO_PASS) -> np.ndarray:
+    """Full output ``[B, N, H, D]`` in float64.  ``q, k, v`` are uint16 bit
+    patterns (dtype BF16 or F16) or float64 arrays (dtype F64), shape [B,N,H,D]."""
+    q, k, v = (_as_input(x, dtype) for x in (q, k, v))
+    if q.ndim != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, N, H, D] shape")
+    B, N, H, D = q.shape
+    out = np.empty((B, N, H, D), dtype=np.float64)
+    rc = _load().oracle_attention(_ptr(q), _ptr(k), _ptr(v), B, N, H, D, float(scale), dtype, mode,
+                                  _ptr(out))
+    if rc:
+        raise RuntimeError(f"oracle_attention failed with code {rc}")
+    return out
+
+
+def attention_rows(q, k, v, scale: float, dtype: int, rows, mode: int = MODE_TWO_PASS) -> np.ndarray:
+    """Selected output rows: ``rows`` holds flat token-head indices
+    ``(b*N + i)*H + h``; returns ``[len(rows), D]`` float64."""
+    q, k, v = (_as_input(x, dtype) for x in (q, k, v))
+    B, N, H, D = q.shape
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    out = np.empty((rows.size, D), dtype=np.float64)
+    rc = _load().oracle_attention_rows(_ptr(q), _ptr(k), _ptr(v), B, N, H, D, float(scale), dtype,
+                                       mode, _ptr(rows), rows.size, _ptr(out))
+    if rc:
+        raise RuntimeError(f"oracle_attention_rows failed with code {rc}")
+    return out
+
+
+def probs(q, k, scale: float, dtype: int, b: int, h: int) -> np.ndarray:
+    """The N x N softmax probability matrix of one (b, h) slice."""
+    q, k = (_as_input(x, dtype) for x in (q, k))
+    B, N, H, D = q.shape
+    P = np.empty((N, N), dtype=np.float64)
+    rc = _load().oracle_attention_probs(_ptr(q), _ptr(k), B, N, H, D, float(scale), dtype, b, h,
+                                        _ptr(P))
+    if rc:
+        raise RuntimeError(f"oracle_attention_probs failed with code {rc}")
+    return P
+
+
+def widen(bits: np.ndarray, dtype: int) -> np.ndarray:
+    """bf16 / f16 bit patterns to float64, exactly."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(bits.shape, dtype=np.float64)
+    rc = _load().oracle_widen(_ptr(bits), bits.size, dtype, _ptr(out))
+    if rc:
+        raise RuntimeError(f"oracle_widen failed with code {rc}")
+    return out
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle runs on."""
+    return int(_load().oracle_num_threads())

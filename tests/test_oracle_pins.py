@@ -1,0 +1,304 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+The oracle computes, per (batch, head), O = softmax(scale * Q K^T) V with no
+mask (hf2q ``src/inference/vision/vit_gpu.rs``: doc of ``vit_attention_gpu``
+and ``vit_attention_scores_gpu``; inferencelayer ``src/vision_gpu.rs``:
+``vis_attn_coop_src`` doc).  Each test below pins it to a closed form, an
+invariant of the definition, a hand-derived fixture, exhaustive conversion
+tables, or an independent library routine, so that a dropped term, a wrong
+sign, a transposed operand or a mixed-up index fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from vit_bidirectional_attention_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_form_cases.txt")
+
+
+def rnd(shape, seed, std=1.0):
+    return np.random.Generator(np.random.PCG64(seed)).standard_normal(size=shape) * std
+
+
+# ---------------------------------------------------------------- conversions
+
+def test_widen_f16_exhaustive_matches_numpy():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.widen(bits, oracle.F16)
+    want = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+
+
+def test_widen_bf16_exhaustive_matches_torch():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.widen(bits, oracle.BF16)
+    want = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+
+
+@pytest.mark.parametrize("dtype", [synth.BF16, synth.F16])
+def test_generator_rounding_is_round_to_nearest_even(dtype):
+    x = rnd(200_000, 5, std=3.0).astype(np.float32)
+    x[:4] = [0.0, -0.0, 1e-8, 65504.0]
+    bits = synth.round_to_bits(x, dtype)
+    tdt = torch.bfloat16 if dtype == synth.BF16 else torch.float16
+    want = torch.from_numpy(x).to(tdt).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bits, want)
+
+
+# ---------------------------------------------------------------- fixtures
+
+def _parse_golden():
+    cases, cur = [], None
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        tok = line.split()
+        if tok[0] == "case":
+            kv = dict(t.split("=") for t in tok[2:])
+            cur = {"name": tok[1], "N": int(kv["N"]), "D": int(kv["D"]), "scale": float(kv["scale"])}
+        elif tok[0] in ("q", "k", "v"):
+            cur[tok[0]] = np.array([float(t) for t in tok[1:]])
+        elif tok[0] == "o":
+            env = {"sig": lambda x: 1.0 / (1.0 + math.exp(-x)), "exp": math.exp}
+            cur["o"] = np.array([eval(t, {"__builtins__": {}}, env) for t in tok[1:]])
+        elif tok[0] == "end":
+            cases.append(cur)
+    return cases
+
+
+GOLDEN_CASES = _parse_golden()
+
+
+@pytest.mark.parametrize("case", GOLDEN_CASES, ids=[c["name"] for c in GOLDEN_CASES])
+@pytest.mark.parametrize("dtype", [oracle.F64, oracle.BF16, oracle.F16])
+def test_hand_derived_closed_forms(case, dtype):
+    N, D = case["N"], case["D"]
+    shape = (1, N, 1, D)
+    q, k, v = (case[n].reshape(shape) for n in "qkv")
+    if dtype != oracle.F64:
+        q, k, v = (synth.round_to_bits(x.astype(np.float32), dtype) for x in (q, k, v))
+    out = oracle.attention(q, k, v, case["scale"], dtype)
+    np.testing.assert_allclose(out.reshape(-1), case["o"], rtol=0, atol=1e-15)
+
+
+def test_golden_file_has_cases():
+    assert len(GOLDEN_CASES) >= 3
+
+
+# ---------------------------------------------------------------- closed forms
+
+@pytest.mark.parametrize("scale", [0.125, 1.0, -3.0, 40.0])
+def test_single_token_returns_v(scale):
+    q, k, v = (rnd((2, 1, 3, 16), s) for s in (1, 2, 3))
+    out = oracle.attention(q, k, v, scale, oracle.F64)
+    assert np.array_equal(out, v)
+
+
+def test_zero_scale_gives_mean_of_v():
+    q, k, v = (rnd((2, 37, 3, 24), s) for s in (4, 5, 6))
+    out = oracle.attention(q, k, v, 0.0, oracle.F64)
+    want = np.broadcast_to(v.mean(axis=1, keepdims=True), v.shape)
+    np.testing.assert_allclose(out, want, rtol=0, atol=1e-14)
+
+
+def test_identical_keys_give_mean_of_v():
+    B, N, H, D = 1, 50, 2, 32
+    q, v = rnd((B, N, H, D), 7), rnd((B, N, H, D), 8)
+    k = np.broadcast_to(rnd((B, 1, H, D), 9), (B, N, H, D)).copy()
+    out = oracle.attention(q, k, v, 0.3, oracle.F64)
+    want = np.broadcast_to(v.mean(axis=1, keepdims=True), v.shape)
+    np.testing.assert_allclose(out, want, rtol=0, atol=1e-14)
+
+
+def test_all_ones_v_gives_ones():
+    q, k = rnd((2, 70, 2, 16), 10, std=2.0), rnd((2, 70, 2, 16), 11, std=2.0)
+    v = np.ones_like(q)
+    out = oracle.attention(q, k, v, 0.25, oracle.F64)
+    np.testing.assert_allclose(out, 1.0, rtol=0, atol=1e-14)
+
+
+def test_two_keys_logistic_form():
+    # N = 2: O_i = sig(s_i0 - s_i1) v_0 + sig(s_i1 - s_i0) v_1 with s = scale * q.k
+    q, k, v = (rnd((1, 2, 1, 8), s) for s in (12, 13, 14))
+    scale = 0.7
+    out = oracle.attention(q, k, v, scale, oracle.F64)[0, :, 0]
+    sig = lambda x: 1.0 / (1.0 + math.exp(-x))
+    for i in range(2):
+        d = scale * (float(q[0, i, 0] @ k[0, 0, 0]) - float(q[0, i, 0] @ k[0, 1, 0]))
+        want = sig(d) * v[0, 0, 0] + sig(-d) * v[0, 1, 0]
+        np.testing.assert_allclose(out[i], want, rtol=0, atol=1e-15)
+
+
+def test_dominant_key_selects_its_value():
+    B, N, H, D = 1, 40, 1, 16
+    q = np.zeros((B, N, H, D)); q[..., 0] = 1.0
+    k = rnd((B, N, H, D), 15) * 0.01
+    k[0, 17, 0, 0] = 100.0
+    v = rnd((B, N, H, D), 16)
+    out = oracle.attention(q, k, v, 1.0, oracle.F64)
+    np.testing.assert_allclose(out[0, :, 0], np.broadcast_to(v[0, 17, 0], (N, D)), rtol=0, atol=1e-30)
+
+
+def test_huge_logits_stay_finite():
+    # the max shift keeps exp in range; without it exp(2000) overflows
+    q, k, v = (rnd((1, 30, 1, 8), s) for s in (17, 18, 19))
+    out = oracle.attention(q, k, v, 500.0, oracle.F64)
+    assert np.all(np.isfinite(out))
+    P = oracle.probs(q, k, 500.0, oracle.F64, 0, 0)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+
+
+def test_all_scores_far_below_zero_stay_finite():
+    # every score near -1000: exp(s) underflows unless the row maximum is subtracted
+    g = np.random.Generator(np.random.PCG64(48))
+    q = np.abs(g.standard_normal((1, 25, 2, 8))) + 1.0
+    k = np.abs(g.standard_normal((1, 25, 2, 8))) + 1.0
+    v = g.standard_normal((1, 25, 2, 8))
+    out = oracle.attention(q, k, v, -80.0, oracle.F64)
+    assert np.all(np.isfinite(out))
+    # the least negative score dominates: compare against the row argmax of q.k scaled
+    P = oracle.probs(q, k, -80.0, oracle.F64, 0, 1)
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    s = -80.0 * np.einsum("id,jd->ij", q[0, :, 1], k[0, :, 1])
+    assert np.array_equal(P.argmax(axis=1), s.argmax(axis=1))
+
+
+# ---------------------------------------------------------------- invariants
+
+def test_probability_rows_sum_to_one_and_produce_out():
+    q, k, v = (rnd((2, 45, 3, 24), s) for s in (20, 21, 22))
+    out = oracle.attention(q, k, v, 0.4, oracle.F64)
+    for b in range(2):
+        for h in range(3):
+            P = oracle.probs(q, k, 0.4, oracle.F64, b, h)
+            assert np.all(P >= 0)
+            np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+            np.testing.assert_allclose(P @ v[b, :, h], out[b, :, h], rtol=0, atol=1e-13)
+
+
+def test_joint_key_value_permutation_invariance():
+    q, k, v = (rnd((2, 33, 2, 16), s) for s in (23, 24, 25))
+    perm = np.random.Generator(np.random.PCG64(26)).permutation(33)
+    a = oracle.attention(q, k, v, 0.5, oracle.F64)
+    b = oracle.attention(q, k[:, perm], v[:, perm], 0.5, oracle.F64)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+def test_query_permutation_permutes_output():
+    q, k, v = (rnd((1, 29, 2, 16), s) for s in (27, 28, 29))
+    perm = np.random.Generator(np.random.PCG64(30)).permutation(29)
+    a = oracle.attention(q, k, v, 0.5, oracle.F64)
+    b = oracle.attention(q[:, perm], k, v, 0.5, oracle.F64)
+    np.testing.assert_allclose(a[:, perm], b, rtol=0, atol=1e-15)
+
+
+def test_affine_in_v():
+    q, k, v = (rnd((1, 31, 2, 8), s) for s in (31, 32, 33))
+    c = rnd((8,), 34)
+    a = oracle.attention(q, k, v, 0.6, oracle.F64)
+    b = oracle.attention(q, k, 2.5 * v + c, 0.6, oracle.F64)
+    np.testing.assert_allclose(b, 2.5 * a + c, rtol=0, atol=1e-13)
+
+
+def test_common_key_shift_leaves_output_unchanged():
+    # K[j] -> K[j] + c shifts every score of row i by scale*q_i.c: softmax ignores it.
+    # Small integers keep every input exact in bf16.
+    g = np.random.Generator(np.random.PCG64(35))
+    q = g.integers(-2, 3, size=(1, 20, 2, 16)).astype(np.float32)
+    k = g.integers(-2, 3, size=(1, 20, 2, 16)).astype(np.float32)
+    v = g.integers(-4, 5, size=(1, 20, 2, 16)).astype(np.float32)
+    c = g.integers(-3, 4, size=(16,)).astype(np.float32)
+    bits = lambda x: synth.round_to_bits(x, synth.BF16)
+    a = oracle.attention(bits(q), bits(k), bits(v), 0.25, oracle.BF16)
+    b = oracle.attention(bits(q), bits(k + c), bits(v), 0.25, oracle.BF16)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+def test_heads_and_batches_are_independent_slices():
+    B, N, H, D = 2, 19, 3, 8
+    q, k, v = (rnd((B, N, H, D), s) for s in (36, 37, 38))
+    full = oracle.attention(q, k, v, 0.9, oracle.F64)
+    for b in range(B):
+        for h in range(H):
+            sl = lambda x: np.ascontiguousarray(x[b:b + 1, :, h:h + 1, :])
+            one = oracle.attention(sl(q), sl(k), sl(v), 0.9, oracle.F64)
+            assert np.array_equal(one[0, :, 0], full[b, :, h])
+
+
+# ---------------------------------------------------------------- library routine
+
+@pytest.mark.parametrize("shape,scale", [((2, 65, 3, 64), 0.125), ((1, 130, 2, 72), 1 / math.sqrt(72)),
+                                         ((3, 17, 1, 80), -0.2), ((1, 5, 4, 16), 2.0)])
+def test_matches_torch_sdpa_float64(shape, scale):
+    q, k, v = (rnd(shape, 40 + s, std=1.5) for s in range(3))
+    out = oracle.attention(q, k, v, scale, oracle.F64)
+    t = lambda x: torch.from_numpy(x).permute(0, 2, 1, 3)  # [B,H,N,D]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), scale=scale)
+    ref = ref.permute(0, 2, 1, 3).numpy()
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- internal consistency
+
+@pytest.mark.parametrize("dtype", [oracle.BF16, oracle.F16])
+def test_formulations_agree_on_tiny(dtype):
+    w = synth.WORKLOADS["tiny"]
+    q, k, v = synth.random_qkv(1, 48, 2, 16, dtype, seed=44)
+    a = oracle.attention(q, k, v, 0.25, dtype, mode=oracle.MODE_TWO_PASS)
+    b = oracle.attention(q, k, v, 0.25, dtype, mode=oracle.MODE_LSE)
+    c = oracle.attention(q, k, v, 0.25, dtype, mode=oracle.MODE_BRUTE)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(a, c, rtol=0, atol=1e-12)
+    assert w.N == 64
+
+
+def test_bits_path_equals_widened_f64_path():
+    q, k, v = synth.random_qkv(2, 40, 3, 24, synth.F16, seed=45)
+    a = oracle.attention(q, k, v, 0.3, oracle.F16)
+    b = oracle.attention(*(oracle.widen(x, oracle.F16) for x in (q, k, v)), 0.3, oracle.F64)
+    assert np.array_equal(a, b)
+
+
+def test_rows_entry_matches_full_output():
+    q, k, v = synth.random_qkv(2, 70, 3, 16, synth.BF16, seed=46)
+    full = oracle.attention(q, k, v, 0.25, oracle.BF16)
+    rows = synth.sample_rows((2, 70, 3), 50, seed=47)
+    part = oracle.attention_rows(q, k, v, 0.25, oracle.BF16, rows)
+    assert np.array_equal(part, full.reshape(-1, 16)[rows])
+
+
+def test_bad_arguments_raise():
+    q = np.zeros((1, 4, 1, 8), dtype=np.uint16)
+    with pytest.raises(RuntimeError):
+        oracle.attention_rows(q, q, q, 1.0, oracle.BF16, np.array([4], dtype=np.int64))
+    with pytest.raises(TypeError):
+        oracle.attention(q.astype(np.float32), q, q, 1.0, oracle.BF16)
+
+
+def test_workload_table_matches_stated_shapes():
+    w = synth.WORKLOADS
+    assert (w["small_vit"].N, w["small_vit"].H, w["small_vit"].D) == (196, 16, 72)
+    assert (w["doc_page"].N, w["doc_page"].D) == (912, 80)
+    assert (w["batched"].B, w["batched"].N, w["batched"].D) == (32, 1024, 64)
+    assert (w["high_res"].B, w["high_res"].N, w["high_res"].D) == (2, 16384, 128)
+    assert w["batched"].flops == 4 * 32 * 16 * 1024 ** 2 * 64
+
+
+def test_rank8_recipe_reaches_logit_std_4():
+    # measured on a reduced-N copy of the high-res recipe (same D, same alpha)
+    w = synth.Workload("hr_small", 1, 2048, 2, 128, synth.BF16, rank8_logit_std=4.0, index=4)
+    q, k, _ = synth.make_qkv(w)
+    qf, kf = (synth.bits_to_float32(x, synth.BF16).astype(np.float64) for x in (q, k))
+    s = np.einsum("nd,md->nm", qf[0, :, 0], kf[0, :, 0]) / math.sqrt(128)
+    assert 3.6 < s.std() < 4.4

@@ -1,0 +1,173 @@
+"""Seeded synthetic attention inputs: the one module both the oracle and the
+CUDA path are fed from.
+
+It holds no attention arithmetic.  It draws Q, K, V as IEEE single-precision
+normals from a seeded PCG64 stream, shapes them as the workloads below
+describe, and rounds them once (round-to-nearest-even) to the storage dtype.
+The result is a set of uint16 bit patterns that the oracle widens exactly to
+double and that the GPU library reads as bf16 / f16.
+
+Workloads (token-major ``[B, N, H, D]`` as they leave a ViT's QKV linear):
+
+- ``tiny``       1 x 64 x 2 x 64, bf16, iid N(0,1)
+- ``small_vit``  1 x 196 x 16 x 72, f16, iid N(0,1)  (14x14 patches, hidden 1152;
+  the SigLIP/Gemma-4V block shape of hf2q ``vit_gpu.rs``)
+- ``doc_page``   1 x 912 x 16 x 80, bf16, Q,K iid N(0, 1.5^2), V iid N(0,1)
+  (the 912-patch page of inferencelayer ``vision_gpu.rs``, module doc)
+- ``batched``    32 x 1024 x 16 x 64, bf16, iid N(0,1)
+- ``high_res``   2 x 16384 x 16 x 128, bf16, Q = Zq + a*Uq*W, K = Zk + a*Uk*W
+  with Z iid N(0,1), U: N x 8 iid N(0,1) per tensor and per (b, h), W: 8 x D
+  with orthonormal rows per (b, h) shared by Q and K, and a = sqrt(sqrt(241)-1)
+  so that a logit q.k/sqrt(D) has variance 1 + (16a^2 + 8a^4)/D = 16 (std 4:
+  a peaky softmax that keeps raising the running maximum); V iid N(0,1).
+
+Every workload uses scale = 1/sqrt(D) and seed 20261202 + its index.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+BF16, F16 = 0, 1
+DTYPE_NAMES = {BF16: "bf16", F16: "f16"}
+SEED_BASE = 20261202
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    N: int
+    H: int
+    D: int
+    dtype: int
+    qk_std: float = 1.0
+    rank8_logit_std: float = 0.0  # 0: iid; >0: shared rank-8 component reaching this logit std
+    index: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def seed(self) -> int:
+        return SEED_BASE + self.index
+
+    @property
+    def flops(self) -> float:
+        """4*B*H*N^2*D: the two contractions QK^T and PV, two flops per MAC."""
+        return 4.0 * self.B * self.H * self.N * self.N * self.D
+
+    @property
+    def io_bytes(self) -> int:
+        """Q, K, V read once and O written once, 2 bytes per element."""
+        return 4 * self.B * self.N * self.H * self.D * 2
+
+    @property
+    def numel(self) -> int:
+        return self.B * self.N * self.H * self.D
+
+
+WORKLOADS = {
+    w.name: w
+    for w in (
+        Workload("tiny", 1, 64, 2, 64, BF16, index=0),
+        Workload("small_vit", 1, 196, 16, 72, F16, index=1),
+        Workload("doc_page", 1, 912, 16, 80, BF16, qk_std=1.5, index=2),
+        Workload("batched", 32, 1024, 16, 64, BF16, index=3),
+        Workload("high_res", 2, 16384, 16, 128, BF16, rank8_logit_std=4.0, index=4),
+    )
+}
+
+
+def round_to_bits(x: np.ndarray, dtype: int) -> np.ndarray:
+    """float32 -> bf16 / f16 bit patterns, round to nearest even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if dtype == F16:
+        return x.astype(np.float16).view(np.uint16)
+    if dtype != BF16:
+        raise ValueError(f"unknown dtype code {dtype}")
+    u = x.view(np.uint32).astype(np.uint64)
+    nan = (u & 0x7F800000) == 0x7F800000
+    nan &= (u & 0x007FFFFF) != 0
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    rounded = np.where(nan, (u >> 16) | 0x40, rounded)
+    return rounded.astype(np.uint16)
+
+
+def bits_to_float32(bits: np.ndarray, dtype: int) -> np.ndarray:
+    """Inverse of :func:`round_to_bits` (exact)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    if dtype == F16:
+        return bits.view(np.float16).astype(np.float32)
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def _rank8_alpha(D: int, logit_std: float) -> float:
+    # logit variance 1 + (16 a^2 + 8 a^4) / D = logit_std^2  ->  a^4 + 2 a^2 - c = 0
+    c = (logit_std * logit_std - 1.0) * D / 8.0
+    a2 = -1.0 + math.sqrt(1.0 + c)
+    return math.sqrt(a2)
+
+
+def make_qkv(w: Workload, seed: int | None = None):
+    """(q, k, v) uint16 bit arrays of shape [B, N, H, D] for workload ``w``."""
+    rng = np.random.Generator(np.random.PCG64(w.seed if seed is None else seed))
+    shape = (w.B, w.N, w.H, w.D)
+
+    def normal(std: float = 1.0) -> np.ndarray:
+        x = rng.standard_normal(size=shape, dtype=np.float32)
+        if std != 1.0:
+            x *= np.float32(std)
+        return x
+
+    if w.rank8_logit_std > 0.0:
+        alpha = np.float32(_rank8_alpha(w.D, w.rank8_logit_std))
+        zq = normal()
+        zk = normal()
+        for b in range(w.B):
+            for h in range(w.H):
+                g = rng.standard_normal(size=(w.D, 8))
+                basis, _ = np.linalg.qr(g)                     # D x 8, orthonormal columns
+                W = basis.T.astype(np.float32)                 # 8 x D, orthonormal rows
+                uq = rng.standard_normal(size=(w.N, 8), dtype=np.float32)
+                uk = rng.standard_normal(size=(w.N, 8), dtype=np.float32)
+                zq[b, :, h, :] += alpha * (uq @ W)
+                zk[b, :, h, :] += alpha * (uk @ W)
+        q, k = zq, zk
+    else:
+        q = normal(w.qk_std)
+        k = normal(w.qk_std)
+    v = normal()
+    return tuple(round_to_bits(x, w.dtype) for x in (q, k, v))
+
+
+def random_qkv(B: int, N: int, H: int, D: int, dtype: int, seed: int, std: float = 1.0):
+    """iid N(0, std^2) inputs for shape sweeps (same recipe, free shape)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for _ in range(3):
+        x = rng.standard_normal(size=(B, N, H, D), dtype=np.float32)
+        if std != 1.0:
+            x *= np.float32(std)
+        out.append(round_to_bits(x, dtype))
+    return tuple(out)
+
+
+def sample_rows(w_or_shape, count: int, seed: int) -> np.ndarray:
+    """``count`` distinct flat token-head row indices ``(b*N + i)*H + h``,
+    always including the first and last row of the tensor."""
+    if isinstance(w_or_shape, Workload):
+        B, N, H = w_or_shape.B, w_or_shape.N, w_or_shape.H
+    else:
+        B, N, H = w_or_shape[:3]
+    total = B * N * H
+    count = min(count, total)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows = rng.choice(total, size=count, replace=False).astype(np.int64)
+    rows[0] = 0
+    if count > 1:
+        rows[-1] = total - 1
+    return np.unique(rows)
