@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark: device-timed attention forward on B200, one JSON line.
+
+A step is one call of ``vitattn_forward`` over one batch of the workload:
+the whole path (Q.K^T, online softmax, P.V, epilogue) in one kernel launch.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+* ``value``: 4*B*H*N^2*D flops per step x steps x ranks / device time of the
+  timed region (CUDA events on the launching stream, max over ranks), TFLOP/s.
+* ``e2e``: the same metric through the host-buffer entry point
+  ``vitattn_forward_host`` (pinned host -> device copies of q, k, v, the
+  kernel, device -> host copy of out, all inside the timed region).
+* ``roofline``: the kernel against the measured dense bf16 tensor peak.
+* ``cpu_baseline``: the fp64 oracle on this host's cores, on a bounded sample
+  of output rows of the same workload, scaled to the same metric.
+
+With ``--gpus N`` (under torchrun) every rank runs the full workload on its
+own GPU with no collective on the data path (the (b, h) units are
+independent): weak scaling; ranks only meet for barriers and the max of the
+timings.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from vit_bidirectional_attention_b200 import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "batched"
+METRIC = "attention fwd TFLOP/s (4·B·H·N²·D) and % of B200 dense BF16 tensor peak"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAK_TFLOPS = 1590.0  # the pool's earlier measurement, used only without MEASURED_PEAKS.json
+DATASHEET_PEAK_TFLOPS = 2250.0
+KERNEL_SOURCES = ["vit_bidirectional_attention_b200/csrc/fwd_kernel.cuh",
+                  "vit_bidirectional_attention_b200/csrc/ptx.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "MEASURED_PEAKS.json"
+    return None, "fallback"
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        data = json.load(f)
+    entry = data.get(workload)
+    if not entry or entry.get("kernel_hash") != kernel_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+
+    FIELDS = ("index,timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.t_start = self.t_stop = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append({"sm": float(parts[2]), "max": float(parts[3]), "reasons": parts[5:10]})
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["sm"] > 0.5 * r["max"]] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        active = set()
+        for r in loaded:
+            for n, flag in zip(names, r["reasons"][1:]):
+                if flag.lower() == "active":
+                    active.add(n)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+                "sm_max_mhz": max(r["max"] for r in loaded),
+                "reasons": sorted(active), "samples": len(loaded)}
+
+
+def cpu_baseline(w, q, k, v, seconds: float):
+    """The fp64 oracle, as it stands, on a bounded sample of output rows."""
+    import oracle
+
+    flops_per_row = 4.0 * w.N * w.D
+    total_rows = w.B * w.N * w.H
+    rows = synth.sample_rows(w, min(64, total_rows), seed=w.seed + 11)
+    t0 = time.perf_counter()
+    oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
+    t_probe = max(time.perf_counter() - t0, 1e-6)
+    want = int(min(total_rows, max(64, len(rows) * seconds / t_probe)))
+    rows = synth.sample_rows(w, want, seed=w.seed + 13)
+    t0 = time.perf_counter()
+    oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
+    dt = time.perf_counter() - t0
+    return {"value": flops_per_row * len(rows) / dt / 1e12, "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} of {total_rows} output rows (seeded), fp64, "
+                      f"{dt:.1f} s on {oracle.num_threads()} threads"}
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args):
+    """The oracle as the reference arm: bounded samples on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+
+    w = synth.WORKLOADS[args.workload]
+    q, k, v = synth.make_qkv(w)
+    total_rows = w.B * w.N * w.H
+    per_step = max(1.0, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
+    rows_probe = synth.sample_rows(w, min(64, total_rows), seed=w.seed + 17)
+    t0 = time.perf_counter()
+    oracle.attention_rows(q, k, v, w.scale, w.dtype, rows_probe)
+    t_probe = max(time.perf_counter() - t0, 1e-6)
+    n_rows = int(min(total_rows, max(32, len(rows_probe) * per_step / t_probe)))
+    flops_per_row = 4.0 * w.N * w.D
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = synth.sample_rows(w, n_rows, seed=w.seed + 1000 + i)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    step_s = sum(times) / len(times)
+    value = flops_per_row * n_rows / step_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "B": w.B, "N": w.N, "H": w.H, "D": w.D,
+                   "input_dtype": synth.DTYPE_NAMES[w.dtype], "scale": w.scale,
+                   "sample_rows_per_step": n_rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{n_rows} of {total_rows} output rows per step (seeded)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import numpy as np
+    import torch
+
+    from vit_bidirectional_attention_b200 import vitattn
+
+    world, rank, local = dist_setup(args)
+    w = synth.WORKLOADS[args.workload]
+    q, k, v = synth.make_qkv(w)
+    tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
+    dev = torch.device("cuda", local if world > 1 else 0)
+
+    def host(bits):
+        return torch.from_numpy(bits.view(np.int16).copy()).view(tdt)
+
+    hq, hk, hv = (host(x) for x in (q, k, v))
+    dq, dk, dv = (x.to(dev) for x in (hq, hk, hv))
+    dout = torch.empty_like(dq)
+    stream = torch.cuda.Stream(dev)
+    sh = stream.cuda_stream
+    L = vitattn.lib()
+
+    def step():
+        rc = L.vitattn_forward(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
+                               w.N, w.H, w.D, w.scale, w.dtype, sh)
+        if rc:
+            raise vitattn.VitAttnError(rc, "vitattn_forward")
+
+    # correctness gate on this exact launch configuration before timing
+    with torch.cuda.stream(stream):
+        rc = vitattn.forward_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
+                                 w.N, w.H, w.D, w.scale, w.dtype, sh, checked=True)
+    if rc:
+        raise vitattn.VitAttnError(rc, "vitattn_forward_checked")
+
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark("t_start")
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    ev1.synchronize()
+    sampler.mark("t_stop")
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+    clocks = sampler.stop()
+    ms_step = ms_total / args.steps
+    tflops = w.flops * args.steps * world / (ms_total * 1e-3) / 1e12
+    per_gpu_tflops = w.flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the host-buffer entry point
+    hq_p, hk_p, hv_p = (x.pin_memory() for x in (hq, hk, hv))
+    hout_p = torch.empty_like(hq).pin_memory()
+    e2e_steps = max(1, args.e2e_steps)
+
+    def e2e_step():
+        rc = L.vitattn_forward_host(hq_p.data_ptr(), hk_p.data_ptr(), hv_p.data_ptr(),
+                                    hout_p.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                    dout.data_ptr(), w.B, w.N, w.H, w.D, w.scale, w.dtype, sh)
+        if rc:
+            raise vitattn.VitAttnError(rc, "vitattn_forward_host")
+
+    for _ in range(2):
+        e2e_step()
+    stream.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    e1.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = w.flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = measured_peaks()
+    if peaks:
+        peak = float(peaks["bf16_tflops"])
+        peak_note = "measured burst dense bf16 (cuBLAS 8192^3), MEASURED_PEAKS.json"
+    else:
+        peak = FALLBACK_PEAK_TFLOPS
+        peak_note = "fallback 1.59 PFLOP/s (pool's earlier measurement)"
+    if w.dtype == synth.F16:
+        peak_note += "; f16 runs at the bf16 rate (same nominal dense figure)"
+
+    result = None
+    if rank == 0:
+        cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline(w, q, k, v, args.cpu_seconds)
+        traffic = committed_traffic(args.workload)
+        result = {
+            "metric": METRIC,
+            "value": tflops,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": synth.DTYPE_NAMES[w.dtype],
+            "data": "synthetic (seeded normals with the workload's shape and distribution)",
+            "config": {
+                "workload": args.workload, "B": w.B, "N": w.N, "H": w.H, "D": w.D,
+                "scale": w.scale, "global_batch": w.B * world,
+                "parallelism": f"independent (b,h) units per GPU x{world}",
+                "l2": (f"inputs {w.io_bytes / 2**20:.0f} MiB > 126 MiB L2, no flush"
+                       if w.io_bytes > L2_BYTES else
+                       f"inputs {w.io_bytes / 2**20:.1f} MiB fit in L2 (warm)"),
+                "flops_per_step": w.flops,
+            },
+            "pct_of_datasheet_peak": 100.0 * per_gpu_tflops / DATASHEET_PEAK_TFLOPS,
+            "roofline": {
+                "bound": "tensor",
+                "achieved": per_gpu_tflops,
+                "peak": peak,
+                "unit": "TFLOP/s",
+                "frac": per_gpu_tflops / peak,
+                "traffic": traffic,
+                "peak_source": peak_note if peaks else "fallback",
+                "kernel": "vitattn::fwd_kernel",
+                "algorithmic_flops_per_launch": w.flops,
+                "algorithmic_bytes_per_launch": w.io_bytes,
+                "achieved_hbm_gbs": w.io_bytes / (ms_step * 1e-3) / 1e9,
+            },
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": 3 * w.numel * 2, "d2h_bytes_per_step": w.numel * 2,
+                    "ms_per_step": e2e_ms / e2e_steps, "entry": "vitattn_forward_host"},
+            "gpu_launches": args.steps * vitattn.launches_per_call(),
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,147 @@
+/*
+ * vitattn.h -- C ABI of libvitattn: the forward pass of non-causal multi-head
+ * scaled-dot-product attention inside a vision-transformer encoder block, on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For every batch b < B and head h < H, with
+ * Q_bh[i,:] = q[b,i,h,:] (likewise K_bh, V_bh):
+ *
+ *     O_bh = softmax(scale * Q_bh K_bh^T) V_bh        (row softmax, no mask)
+ *
+ * written to out[b,i,h,:].  Sources: hf2q "src/inference/vision/vit_gpu.rs",
+ * doc of `vit_attention_gpu` (scores, softmax, P.V; inputs and output
+ * seq-major [batch, num_heads, head_dim]; no mask because a ViT is
+ * bidirectional) and of `vit_attention_scores_gpu` (the caller's scale is
+ * applied as given, with no implicit 1/sqrt(head_dim)); inferencelayer
+ * "src/vision_gpu.rs", doc of `vis_attn_coop_src` (Q.K^T and P.V as GEMMs
+ * with an online softmax that rescales the running output); hanzo-ml
+ * "src/vulkan_backend.rs", `flash_attn_gpu` (the (q, k, v, sizes, scale)
+ * calling shape and argument checks before dispatch).
+ *
+ * Layout.  q, k, v and out are dense, token-major [B, N, H, D] tensors with D
+ * contiguous: element (b, i, h, d) at ((b*N + i)*H + h)*D + d.  That is the
+ * layout a QKV linear produces once its output is split into three.
+ * Lq = Lk = N (self-attention).  out has the dtype of the inputs; products
+ * and sums accumulate in fp32, probabilities are rounded to the input dtype
+ * before the P.V product.
+ *
+ * Ownership.  The caller owns every buffer.  The library allocates no device
+ * memory, keeps no reference to any buffer after a call returns, and never
+ * frees caller memory.  out must not overlap q, k or v.
+ *
+ * Streams and errors.  Calls enqueue work on `stream` and return without
+ * synchronising (except vitattn_forward_checked).  Every argument is checked
+ * before anything is enqueued; a failed check returns a negative status and
+ * enqueues nothing.  A CUDA error raised while enqueueing returns
+ * VITATTN_ERR_CUDA (its cudaError_t value via vitattn_last_cuda_error()).
+ * Errors that happen later on the device surface through the stream, as for
+ * any CUDA kernel.  Every internal wait of the kernel is bounded in time; a
+ * wait that runs out ends the kernel early and records VITATTN_ERR_TIMEOUT in
+ * a device status word, which vitattn_forward_checked reports.
+ *
+ * Thread safety.  Calls may come from several host threads; each call
+ * launches on its own stream argument.
+ */
+#ifndef VITATTN_H
+#define VITATTN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VITATTN_API __attribute__((visibility("default")))
+#else
+#define VITATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream.  NULL means the legacy default stream. */
+typedef struct CUstream_st* vitattn_stream_t;
+
+/* Element type of q, k, v and out. */
+enum vitattn_dtype {
+    VITATTN_BF16 = 0, /* bfloat16 */
+    VITATTN_F16 = 1   /* IEEE binary16 */
+};
+
+/* Return codes.  0 is success; every error is negative. */
+enum vitattn_status {
+    VITATTN_OK = 0,
+    VITATTN_ERR_NULL = -1,    /* a required pointer is NULL */
+    VITATTN_ERR_DIM = -2,     /* B, N or H < 1, or a size or offset would overflow */
+    VITATTN_ERR_HEADDIM = -3, /* D unsupported: needs 16 <= D <= 128 and D % 8 == 0 */
+    VITATTN_ERR_DTYPE = -4,   /* dtype is not a vitattn_dtype */
+    VITATTN_ERR_ALIGN = -5,   /* a tensor pointer is not 16-byte aligned */
+    VITATTN_ERR_ALIAS = -6,   /* out overlaps q, k or v */
+    VITATTN_ERR_CUDA = -7,    /* the CUDA runtime or driver returned an error */
+    VITATTN_ERR_TIMEOUT = -8, /* a bounded in-kernel wait ran out (checked entry only) */
+    VITATTN_ERR_SCALE = -9,   /* scale is NaN or infinite */
+    VITATTN_ERR_DEVICE = -10  /* the current device is not an sm_100 GPU */
+};
+
+/*
+ * vitattn_forward -- out = softmax(scale * Q K^T) V per (batch, head).
+ *   q, k, v  device pointers, [B, N, H, D] of `dtype`, 16-byte aligned.
+ *   out      device pointer, [B, N, H, D] of `dtype`, 16-byte aligned,
+ *            not overlapping q, k or v.  Every element is written.
+ *   B, N, H  batch, tokens per sequence, heads (all >= 1).
+ *   D        head dimension: 16 <= D <= 128, D % 8 == 0.
+ *   scale    multiplies Q K^T as given (pass 1/sqrt(D) for a standard ViT).
+ *   dtype    VITATTN_BF16 or VITATTN_F16.
+ *   stream   stream to launch on.
+ * Launches exactly one kernel on the current CUDA device and returns.
+ */
+VITATTN_API int vitattn_forward(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
+                    int64_t H, int64_t D, float scale, int dtype, vitattn_stream_t stream);
+
+/*
+ * vitattn_forward_checked -- vitattn_forward, then a stream synchronisation
+ * and a read of the kernel's status word.  Returns VITATTN_ERR_TIMEOUT when a
+ * bounded in-kernel wait ran out, VITATTN_ERR_CUDA when the stream reported
+ * an error.  Meant for tests and debugging: it blocks the calling thread.
+ */
+VITATTN_API int vitattn_forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B,
+                            int64_t N, int64_t H, int64_t D, float scale, int dtype,
+                            vitattn_stream_t stream);
+
+/*
+ * vitattn_forward_host -- the same operation from HOST buffers: enqueues the
+ * copies hq->dq, hk->dk, hv->dv, the kernel, and dout->hout, in that order,
+ * on `stream`, and returns without synchronising.  The caller synchronises
+ * the stream before reading hout.  Host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous; the
+ * device buffers dq, dk, dv, dout are caller-owned staging with the same
+ * requirements as in vitattn_forward.  All eight pointers are required.
+ */
+VITATTN_API int vitattn_forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq,
+                         void* dk, void* dv, void* dout, int64_t B, int64_t N, int64_t H,
+                         int64_t D, float scale, int dtype, vitattn_stream_t stream);
+
+/*
+ * vitattn_check_args -- the argument checks of vitattn_forward, alone: no
+ * CUDA call is made, so it runs on a machine without a GPU.  Returns
+ * VITATTN_OK or the status vitattn_forward would return for these arguments
+ * before touching the device.
+ */
+VITATTN_API int vitattn_check_args(const void* q, const void* k, const void* v, const void* out, int64_t B,
+                       int64_t N, int64_t H, int64_t D, float scale, int dtype);
+
+/* Static text for a status code ("unknown status" for anything else). */
+VITATTN_API const char* vitattn_strerror(int status);
+
+/* The cudaError_t of the most recent VITATTN_ERR_CUDA on the calling thread (0 if none). */
+VITATTN_API int vitattn_last_cuda_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+VITATTN_API int vitattn_version(void);
+
+/* Kernel launches one vitattn_forward call makes (for launch accounting). */
+VITATTN_API int vitattn_launches_per_call(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VITATTN_H */

@@ -1,0 +1,102 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and its argument checks return the documented codes before any
+CUDA call (hanzo-ml ``src/vulkan_backend.rs``, ``flash_attn_gpu``: sizes are
+checked before dispatch; hf2q ``src/inference/vision/vit_gpu.rs``,
+``vit_attention_scores_gpu`` "# Errors": zero dims are rejected)."""
+import os
+import re
+import subprocess
+
+import pytest
+
+from vit_bidirectional_attention_b200 import vitattn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vitattn.h")
+
+A = 1 << 20  # fake, 16-byte aligned "device" addresses: nothing is dereferenced
+BYTES = 1 * 64 * 2 * 64 * 2
+Q, K, V, O = A, A + 4 * BYTES, A + 8 * BYTES, A + 12 * BYTES
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"VITATTN_API\s+[\w\s\*]*?\b(vitattn_\w+)\s*\(", text)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    names = header_functions()
+    assert "vitattn_forward" in names and len(names) >= 8
+    L = vitattn.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", vitattn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (vitattn_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_header_enum_values_match_binding():
+    text = open(HEADER).read()
+    for name, val in re.findall(r"(VITATTN_(?:OK|ERR_\w+))\s*=\s*(-?\d+)", text):
+        assert vitattn.STATUS_NAMES[int(val)] == name
+    assert re.search(r"VITATTN_BF16\s*=\s*0", text) and re.search(r"VITATTN_F16\s*=\s*1", text)
+
+
+def test_version_and_launch_count():
+    assert vitattn.version() == 10000
+    assert vitattn.launches_per_call() == 1
+
+
+def ok_args(**kw):
+    a = dict(q=Q, k=K, v=V, out=O, B=1, N=64, H=2, D=64, scale=0.125, dtype=vitattn.BF16)
+    a.update(kw)
+    return a
+
+
+def check(**kw):
+    a = ok_args(**kw)
+    return vitattn.check_args(a["q"], a["k"], a["v"], a["out"], a["B"], a["N"], a["H"], a["D"],
+                              a["scale"], a["dtype"])
+
+
+def test_valid_arguments_pass():
+    assert check() == 0
+    for D in (16, 24, 64, 72, 80, 128):
+        assert check(D=D) == 0, D
+    assert check(dtype=vitattn.F16, scale=-2.0) == 0
+    assert check(scale=0.0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(k=0), -1), (dict(v=0), -1), (dict(out=0), -1),
+    (dict(B=0), -2), (dict(N=0), -2), (dict(H=0), -2), (dict(N=-5), -2),
+    (dict(N=2**31), -2), (dict(B=2**40), -2),
+    (dict(D=8), -3), (dict(D=136), -3), (dict(D=70), -3), (dict(D=0), -2),
+    (dict(dtype=2), -4), (dict(dtype=-1), -4),
+    (dict(q=Q + 8), -5), (dict(out=O + 2), -5),
+    (dict(out=Q), -6), (dict(out=K + 16), -6), (dict(out=V - 16), -6),
+    (dict(scale=float("nan")), -9), (dict(scale=float("inf")), -9),
+])
+def test_argument_errors(kw, code):
+    assert check(**kw) == code
+    assert vitattn.strerror(code) not in ("ok", "unknown status")
+
+
+def test_forward_rejects_bad_arguments_before_any_cuda_call():
+    # these return from the checks, so they are safe on a machine without a GPU
+    assert vitattn.forward_ptr(0, K, V, O, 1, 64, 2, 64, 0.125, 0) == -1
+    assert vitattn.forward_ptr(Q, K, V, O, 1, 64, 2, 60, 0.125, 0) == -3
+    assert vitattn.forward_ptr(Q, K, V, Q, 1, 64, 2, 64, 0.125, 0) == -6
+    assert vitattn.forward_host_ptr(0, 1, 1, 1, Q, K, V, O, 1, 64, 2, 64, 0.125, 0) == -1
+
+
+def test_strerror_unknown():
+    assert vitattn.strerror(12345) == "unknown status"
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(vitattn, "_lib", None)
+    monkeypatch.setattr(vitattn, "LIB_PATH", "/nonexistent/libvitattn.so")
+    with pytest.raises(ImportError):
+        vitattn.lib()

@@ -1,0 +1,230 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Tolerance for every floating-point comparison: max |O_gpu - O_ref| <= 1e-2
+and ||O_gpu - O_ref||_F / ||O_ref||_F <= 4e-3, with O_ref the oracle on the
+same bf16/f16-rounded inputs.  The operation is O = softmax(scale Q K^T) V
+per (batch, head), no mask (hf2q ``src/inference/vision/vit_gpu.rs``, doc of
+``vit_attention_gpu``).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from vit_bidirectional_attention_b200 import synth, vitattn
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+REL_FROB = 4e-3
+
+
+def torch_dtype(dtype):
+    import torch
+
+    return torch.bfloat16 if dtype == synth.BF16 else torch.float16
+
+
+def to_dev(bits, dtype):
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16).copy())
+    return t.view(torch_dtype(dtype)).cuda()
+
+
+def from_dev(t, dtype):
+    import torch
+
+    bits = t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return synth.bits_to_float32(bits, dtype).astype(np.float64)
+
+
+def run_gpu(q, k, v, scale, dtype):
+    tq, tk, tv = (to_dev(x, dtype) for x in (q, k, v))
+    out = vitattn.forward(tq, tk, tv, scale=scale, checked=True)
+    return from_dev(out, dtype)
+
+
+def errors(got, ref):
+    max_abs = float(np.max(np.abs(got - ref)))
+    rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    return max_abs, rel
+
+
+def assert_close(got, ref, what=""):
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    max_abs, rel = errors(got, ref)
+    assert max_abs <= MAX_ABS and rel <= REL_FROB, f"{what}: max_abs={max_abs:.3e} rel_frob={rel:.3e}"
+
+
+# ------------------------------------------------------------------ the workloads
+
+@pytest.mark.parametrize("name", ["tiny", "small_vit", "doc_page"])
+def test_workload_full_parity(cuda_device, name):
+    w = synth.WORKLOADS[name]
+    q, k, v = synth.make_qkv(w)
+    got = run_gpu(q, k, v, w.scale, w.dtype)
+    ref = oracle.attention(q, k, v, w.scale, w.dtype)
+    assert_close(got, ref, name)
+
+
+@pytest.mark.parametrize("name,rows", [("batched", 4096), ("high_res", 1536)])
+def test_workload_sampled_parity_at_full_size(cuda_device, name, rows):
+    """Full-size launch (the configuration the benchmark times); the oracle
+    recomputes a seeded sample of output rows, first and last row included."""
+    w = synth.WORKLOADS[name]
+    q, k, v = synth.make_qkv(w)
+    got = run_gpu(q, k, v, w.scale, w.dtype).reshape(-1, w.D)
+    idx = synth.sample_rows(w, rows, seed=w.seed + 7)
+    ref = oracle.attention_rows(q, k, v, w.scale, w.dtype, idx)
+    assert_close(got[idx], ref, name)
+    # property at any size: every row is a convex combination of V rows, so
+    # each output coordinate lies inside [min_j V, max_j V] of its head
+    vf = synth.bits_to_float32(v, w.dtype).astype(np.float64)
+    vmin = vf.min(axis=1, keepdims=True)
+    vmax = vf.max(axis=1, keepdims=True)
+    g4 = got.reshape(w.B, w.N, w.H, w.D)
+    tol = 1e-2
+    assert np.all(g4 >= vmin - tol) and np.all(g4 <= vmax + tol)
+
+
+# ------------------------------------------------------------------ shape sweep
+
+SWEEP_N = [1, 2, 63, 64, 65, 127, 128, 129, 196, 255, 256, 257, 384, 912, 1024]
+
+
+@pytest.mark.parametrize("N", SWEEP_N)
+@pytest.mark.parametrize("D", [64, 80, 128])
+def test_sweep_tokens(cuda_device, N, D):
+    q, k, v = synth.random_qkv(1, N, 2, D, synth.BF16, seed=1000 + N * 7 + D)
+    scale = 1.0 / math.sqrt(D)
+    assert_close(run_gpu(q, k, v, scale, synth.BF16), oracle.attention(q, k, v, scale, synth.BF16),
+                 f"N={N} D={D}")
+
+
+@pytest.mark.parametrize("dtype", [synth.BF16, synth.F16])
+@pytest.mark.parametrize("D", [16, 24, 32, 40, 48, 56, 64, 72, 80, 88, 96, 104, 112, 120, 128])
+@pytest.mark.parametrize("N", [1, 129, 257])
+def test_sweep_head_dims(cuda_device, dtype, D, N):
+    q, k, v = synth.random_qkv(1, N, 3, D, dtype, seed=2000 + N * 131 + D * 3 + dtype)
+    scale = 1.0 / math.sqrt(D)
+    assert_close(run_gpu(q, k, v, scale, dtype), oracle.attention(q, k, v, scale, dtype),
+                 f"N={N} D={D} dtype={dtype}")
+
+
+def test_many_batches_and_heads(cuda_device):
+    q, k, v = synth.random_qkv(3, 200, 5, 72, synth.F16, seed=3001)
+    assert_close(run_gpu(q, k, v, 0.1, synth.F16), oracle.attention(q, k, v, 0.1, synth.F16))
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.3, 1.0, 2.5])
+def test_scales(cuda_device, scale):
+    q, k, v = synth.random_qkv(1, 300, 2, 64, synth.BF16, seed=3002)
+    assert_close(run_gpu(q, k, v, scale, synth.BF16), oracle.attention(q, k, v, scale, synth.BF16),
+                 f"scale={scale}")
+
+
+def test_peaky_logits_rescale_path(cuda_device):
+    """Logit std ~4 (high-res recipe at reduced N): the running max keeps rising."""
+    w = synth.Workload("peaky", 1, 2048, 4, 128, synth.BF16, rank8_logit_std=4.0, index=4)
+    q, k, v = synth.make_qkv(w)
+    assert_close(run_gpu(q, k, v, w.scale, w.dtype), oracle.attention(q, k, v, w.scale, w.dtype))
+
+
+def test_increasing_logits_force_rescale_every_block(cuda_device):
+    # key j has logit ~ j/8 along q: the row max grows by ~16 per 128-key block
+    N, D = 1024, 64
+    q = np.zeros((1, N, 1, D), np.float32); q[..., 0] = 1.0
+    k = np.zeros((1, N, 1, D), np.float32); k[0, :, 0, 0] = np.arange(N) / 8.0
+    v = np.random.Generator(np.random.PCG64(3003)).standard_normal((1, N, 1, D)).astype(np.float32)
+    q, k, v = (synth.round_to_bits(x, synth.BF16) for x in (q, k, v))
+    assert_close(run_gpu(q, k, v, 1.0, synth.BF16), oracle.attention(q, k, v, 1.0, synth.BF16))
+
+
+# ------------------------------------------------------------------ invariants on GPU output
+
+def test_single_token_returns_v_exactly(cuda_device):
+    q, k, v = synth.random_qkv(4, 1, 3, 80, synth.BF16, seed=3004)
+    got = run_gpu(q, k, v, 0.11, synth.BF16)
+    assert np.array_equal(got, synth.bits_to_float32(v, synth.BF16).astype(np.float64))
+
+
+def test_all_ones_v(cuda_device):
+    q, k, _ = synth.random_qkv(1, 700, 2, 64, synth.BF16, seed=3005, std=2.0)
+    v = synth.round_to_bits(np.ones((1, 700, 2, 64), np.float32), synth.BF16)
+    got = run_gpu(q, k, v, 0.125, synth.BF16)
+    assert np.max(np.abs(got - 1.0)) <= MAX_ABS
+
+
+def test_identical_keys_and_zero_scale_give_mean_of_v(cuda_device):
+    q, k, v = synth.random_qkv(1, 333, 2, 64, synth.BF16, seed=3006)
+    k = np.ascontiguousarray(np.broadcast_to(k[:, :1], k.shape))
+    vf = synth.bits_to_float32(v, synth.BF16).astype(np.float64)
+    mean = np.broadcast_to(vf.mean(axis=1, keepdims=True), vf.shape)
+    assert_close(run_gpu(q, k, v, 0.125, synth.BF16), mean, "identical keys")
+    q2, k2, _ = synth.random_qkv(1, 333, 2, 64, synth.BF16, seed=3007)
+    assert_close(run_gpu(q2, k2, v, 0.0, synth.BF16), mean, "zero scale")
+
+
+def test_joint_key_value_permutation(cuda_device):
+    q, k, v = synth.random_qkv(1, 500, 2, 64, synth.BF16, seed=3008)
+    perm = np.random.Generator(np.random.PCG64(3009)).permutation(500)
+    a = run_gpu(q, k, v, 0.125, synth.BF16)
+    b = run_gpu(q, np.ascontiguousarray(k[:, perm]), np.ascontiguousarray(v[:, perm]), 0.125,
+                synth.BF16)
+    assert_close(b, a, "permuted")
+
+
+def test_bitwise_deterministic(cuda_device):
+    w = synth.WORKLOADS["doc_page"]
+    q, k, v = synth.make_qkv(w)
+    a = run_gpu(q, k, v, w.scale, w.dtype)
+    b = run_gpu(q, k, v, w.scale, w.dtype)
+    assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------ entry points
+
+def test_side_stream_and_preallocated_out(cuda_device):
+    import torch
+
+    w = synth.WORKLOADS["small_vit"]
+    q, k, v = synth.make_qkv(w)
+    tq, tk, tv = (to_dev(x, w.dtype) for x in (q, k, v))
+    out = torch.full_like(tq, float("nan"))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        vitattn.forward(tq, tk, tv, out=out, scale=w.scale, stream=s)
+    s.synchronize()
+    assert_close(from_dev(out, w.dtype), oracle.attention(q, k, v, w.scale, w.dtype))
+
+
+def test_host_buffer_entry_matches(cuda_device):
+    import torch
+
+    w = synth.WORKLOADS["doc_page"]
+    q, k, v = synth.make_qkv(w)
+    tdt = torch_dtype(w.dtype)
+    hosts = [torch.from_numpy(x.view(np.int16).copy()).view(tdt).pin_memory() for x in (q, k, v)]
+    hout = torch.empty_like(hosts[0]).pin_memory()
+    dq, dk, dv, dout = (torch.empty(q.shape, dtype=tdt, device="cuda") for _ in range(4))
+    s = torch.cuda.current_stream()
+    rc = vitattn.forward_host_ptr(*(h.data_ptr() for h in hosts), hout.data_ptr(), dq.data_ptr(),
+                                  dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B, w.N, w.H,
+                                  w.D, w.scale, w.dtype, s.cuda_stream)
+    assert rc == 0
+    s.synchronize()
+    got = from_dev(hout, w.dtype)
+    assert_close(got, oracle.attention(q, k, v, w.scale, w.dtype))
+
+
+def test_errors_on_device_do_not_launch(cuda_device):
+    import torch
+
+    t = torch.zeros((1, 64, 2, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(vitattn.VitAttnError) as e:
+        vitattn.forward(t, t, t, out=t)
+    assert e.value.status == -6
+    assert vitattn.forward_ptr(t.data_ptr() + 2, t.data_ptr(), t.data_ptr(), t.data_ptr() + 4096,
+                               1, 1, 1, 64, 1.0, 0) == -5

@@ -1,0 +1,576 @@
+// fwd_kernel.cuh -- sm_100a forward kernel of non-causal multi-head attention.
+//
+// One CTA owns one (batch b, head h) pair and up to two 128-row query tiles of
+// it (256 query rows).  K and V stream through a shared-memory ring in blocks
+// of 128 keys.  Per key block j and query tile t:
+//
+//   S_t   = Q_t K_j^T                    tcgen05.mma, A = Q (smem), B = K (smem), f32 in TMEM
+//   P_t   = exp2(S_t * c - m_t)          softmax warpgroup t, one thread per query row,
+//                                        c = scale*log2(e); P rounded to the input dtype
+//                                        and written back into TMEM over S_t
+//   O_t  += P_t V_j                      tcgen05.mma, A = P (TMEM), B = V (smem), f32 in TMEM
+//
+// with the running row maximum m_t, the row sum l_t and the rescaling of O_t
+// kept exact in the online-softmax sense: O and l are always relative to the
+// same (possibly stale) maximum, so the result is O/l at the end.  This is the
+// online-softmax GEMM pair of inferencelayer "src/vision_gpu.rs" (doc of
+// `vis_attn_coop_src`: "The obstacle, and the way round it"), except that the
+// running output lives in tensor memory instead of being spilled to shared
+// memory, and that it is only rescaled when a row maximum grows by more than
+// 2^8 (the result is unchanged; probabilities stay <= 256, which bf16 and f16
+// hold).  Keys past N are masked to probability 0 (same page, "Keys past the
+// span ... are masked to zero probability").
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for query tile 0 (TMEM lanes 0..127 through warp%4)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer (one lane) and TMEM allocator (whole warp)
+//   warp  9    MMA issuer (one lane)
+//
+// Tensor memory (512 columns x 128 lanes x 32 bit):
+//   [  0,128)  S_0, later P_0 (16-bit pairs in the first 64 columns)
+//   [128,256)  S_1 / P_1
+//   [256,384)  O_0 (DP columns used)
+//   [384,512)  O_1
+//
+// Shared memory: Q_0, Q_1 and a ring of kStages K/V slots, each a 128 x DP
+// tile stored as column chunks of 64 / 32 / 16 elements (SW128 / SW64 / SW32
+// swizzle, exactly as TMA writes them and as the MMA descriptors read them).
+// DP is D rounded up to a multiple of 16; TMA zero-fills columns D..DP-1.
+//
+// Every wait is bounded by a time limit.  On expiry the kernel records a
+// status code in g_vitattn_status, raises a CTA-wide abort flag that every
+// other waiter polls, drains its own in-flight TMA copies and MMAs, frees its
+// tensor memory and exits.
+#pragma once
+
+#include <cuda.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+// Kernel status word (this header is compiled into exactly one translation
+// unit): 0, or a timeout code from a bounded in-kernel wait.
+__device__ unsigned int g_vitattn_status = 0;
+
+namespace vitattn {
+
+constexpr int kTileRows = 128;    // query rows per tile = TMEM lanes
+constexpr int kBlockKeys = 128;   // keys per K/V block
+constexpr int kTilesPerCta = 2;
+constexpr int kStages = 4;        // K/V ring slots (K_j, V_j, K_j+1, V_j+1)
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
+
+// Barrier indices inside the barrier array.
+constexpr int kBarQFull = 0;                         // [2]
+constexpr int kBarKvFull = 2;                        // [kStages]
+constexpr int kBarKvEmpty = kBarKvFull + kStages;    // [kStages]
+constexpr int kBarSFull = kBarKvEmpty + kStages;     // [2]
+constexpr int kBarPFull = kBarSFull + 2;             // [2]
+constexpr int kBarOFull = kBarPFull + 2;             // [2]
+constexpr int kBarDrain = kBarOFull + 2;             // [1]
+constexpr int kNumBars = kBarDrain + 1;
+
+// Status codes written to g_vitattn_status (0 = fine).
+constexpr unsigned kStatusTimeoutBase = 0x100;  // + site id
+
+// Test-only flag: the producer skips its first V load so that the consumer's
+// bounded wait runs out (exercises the timeout path without a fault).
+constexpr int kFlagSkipFirstVLoad = 1;
+
+// ---------------------------------------------------------------- column chunks
+
+__host__ __device__ constexpr int chunk_count(int dp) {
+    return dp / 64 + ((dp % 64) >= 32 ? 1 : 0) + ((dp % 32) != 0 ? 1 : 0);
+}
+__host__ __device__ constexpr int chunk_width(int dp, int c) {
+    return c < dp / 64 ? 64 : ((c == dp / 64 && (dp % 64) >= 32) ? 32 : 16);
+}
+__host__ __device__ constexpr int chunk_col(int dp, int c) {
+    int col = 0;
+    for (int i = 0; i < c; ++i) col += chunk_width(dp, i);
+    return col;
+}
+__host__ __device__ constexpr int width_class(int w) { return w == 64 ? 0 : (w == 32 ? 1 : 2); }
+// tcgen05 shared-memory descriptor layout codes: SW128 = 2, SW64 = 4, SW32 = 6.
+__host__ __device__ constexpr uint32_t swizzle_code(int w) { return w == 64 ? 2u : (w == 32 ? 4u : 6u); }
+
+__host__ __device__ constexpr int tile_bytes(int dp) { return kTileRows * dp * 2; }
+__host__ __device__ constexpr int smem_bytes(int dp) {
+    return (kTilesPerCta + kStages) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
+}
+
+struct alignas(64) FwdParams {
+    CUtensorMap maps[3][3];  // [q, k, v][width class 64 / 32 / 16]
+    void* out;
+    int B, N, H, D;
+    int n_qpairs;   // ceil(N / 256): CTAs per (b, h)
+    int n_kblocks;  // ceil(N / 128)
+    float scale_log2;
+    int flags;
+    unsigned long long timeout_ns;
+};
+
+// ---------------------------------------------------------------- descriptors
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading and
+// stride byte offsets (16-byte units), fixed version 1 at bit 46, layout code
+// at bits 61..63.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                          uint32_t layout) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+
+// Instruction descriptor, kind::f16: f32 accumulator, A and B both bf16 (1) or
+// both f16 (0), A K-major, B K-major (0) or MN-major (1), N >> 3, M >> 4.
+__host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int n, bool b_mn_major) {
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(kTileRows >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- bounded waits
+
+__device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned site) {
+    *abort_flag = 1;
+    atomicCAS(&g_vitattn_status, 0u, kStatusTimeoutBase + site);
+}
+
+// One thread waits for the phase of `parity`; false on abort or timeout.
+__device__ __noinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                      uint64_t timeout_ns, unsigned site) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (ptx::globaltimer_ns() - t0 > timeout_ns) {
+            raise_abort(abort_flag, site);
+            return false;
+        }
+    }
+}
+
+// Wait that ignores the abort flag, for draining in-flight work before exit.
+__device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::globaltimer_ns() - t0 > timeout_ns) return false;
+    }
+    return true;
+}
+
+// A whole warp waits; the outcome is uniform across the warp.
+__device__ __noinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       uint64_t timeout_ns, unsigned site) {
+    bool done = ptx::mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (true) {
+        if (!done) done = ptx::mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, done)) return true;
+        int give_up = 0;
+        if ((threadIdx.x & 31) == 0) {
+            if (*abort_flag) {
+                give_up = 1;
+            } else if (ptx::globaltimer_ns() - t0 > timeout_ns) {
+                raise_abort(abort_flag, site);
+                give_up = 1;
+            }
+        }
+        if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+    }
+}
+
+// ---------------------------------------------------------------- softmax pieces
+
+// Row extreme of the raw scores in the direction that maximises c * s:
+// max for c >= 0, min for c < 0.  Masked columns (>= valid) are skipped.
+template <bool kPartial>
+__device__ __forceinline__ float row_extreme(const float (&s)[kBlockKeys], int valid, bool neg) {
+    float a = neg ? INFINITY : -INFINITY, b2 = a;
+    if (!neg) {
+#pragma unroll
+        for (int c = 0; c < kBlockKeys; c += 2) {
+            if (!kPartial || c < valid) a = fmaxf(a, s[c]);
+            if (!kPartial || c + 1 < valid) b2 = fmaxf(b2, s[c + 1]);
+        }
+        return fmaxf(a, b2);
+    }
+#pragma unroll
+    for (int c = 0; c < kBlockKeys; c += 2) {
+        if (!kPartial || c < valid) a = fminf(a, s[c]);
+        if (!kPartial || c + 1 < valid) b2 = fminf(b2, s[c + 1]);
+    }
+    return fminf(a, b2);
+}
+
+// p = 2^(c*s - m) for the block, packed to 16-bit pairs; returns sum of p (f32).
+template <bool kPartial, bool kBF16>
+__device__ __forceinline__ float exp_and_pack(const float (&s)[kBlockKeys], int valid, float c2,
+                                              float neg_m, uint32_t (&pk)[kBlockKeys / 2]) {
+    float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < kBlockKeys; c += 2) {
+        float p0 = ptx::ex2(fmaf(s[c], c2, neg_m));
+        float p1 = ptx::ex2(fmaf(s[c + 1], c2, neg_m));
+        if (kPartial) {
+            p0 = c < valid ? p0 : 0.f;
+            p1 = c + 1 < valid ? p1 : 0.f;
+        }
+        l0 += p0;
+        l1 += p1;
+        pk[c / 2] = ptx::pack2<kBF16>(p0, p1);
+    }
+    return l0 + l1;
+}
+
+// Multiply this thread's row of O (DP columns of TMEM at tO) by alpha.
+template <int DP>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll
+    for (int c = 0; c + 32 <= DP; c += 32) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tO + c, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+        ptx::tmem_st32(tO + c, r);
+    }
+    if (DP % 32) {
+        constexpr int c = DP - 16;
+        uint32_t r[16];
+        ptx::tmem_ld16(tO + c, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+        ptx::tmem_st16(tO + c, r);
+    }
+}
+
+// O / l for this thread's row, converted and stored with 16-byte stores.
+template <int DP, bool kBF16>
+__device__ __forceinline__ void store_row(uint32_t tO, float inv_l, uint8_t* orow, bool row_ok,
+                                          int D) {
+#pragma unroll
+    for (int c = 0; c + 32 <= DP; c += 32) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tO + c, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w[i] = ptx::pack2<kBF16>(__uint_as_float(r[8 * g + 2 * i]) * inv_l,
+                                         __uint_as_float(r[8 * g + 2 * i + 1]) * inv_l);
+            const int col = c + 8 * g;
+            if (row_ok && col + 8 <= D) ptx::st_global_v4(orow + 2 * col, w[0], w[1], w[2], w[3]);
+        }
+    }
+    if (DP % 32) {
+        constexpr int c = DP - 16;
+        uint32_t r[16];
+        ptx::tmem_ld16(tO + c, r);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w[i] = ptx::pack2<kBF16>(__uint_as_float(r[8 * g + 2 * i]) * inv_l,
+                                         __uint_as_float(r[8 * g + 2 * i + 1]) * inv_l);
+            const int col = c + 8 * g;
+            if (row_ok && col + 8 <= D) ptx::st_global_v4(orow + 2 * col, w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- the kernel
+
+template <int DP, bool kBF16>
+__global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
+    constexpr int TILE = tile_bytes(DP);
+    constexpr int NCH = chunk_count(DP);
+    static_assert(DP % 16 == 0 && DP >= 16 && DP <= 128, "head dim padding");
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* const base_ptr = smem_raw + (base - raw);
+    const uint32_t sQ = base;
+    const uint32_t sKV = base + kTilesPerCta * TILE;
+    const uint32_t sBar = base + (kTilesPerCta + kStages) * TILE;
+    uint32_t* const tmem_holder =
+        reinterpret_cast<uint32_t*>(base_ptr + (kTilesPerCta + kStages) * TILE + kNumBars * 8);
+    volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    auto bar = [&](int i) -> uint32_t { return sBar + 8u * (uint32_t)i; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // work item -> (b, h, query-tile pair); CTAs of one (b, h) are adjacent so
+    // they share K/V through L2.
+    const int qpair = blockIdx.x % p.n_qpairs;
+    const int bh = blockIdx.x / p.n_qpairs;
+    const int h = bh % p.H;
+    const int b = bh / p.H;
+    const int q0 = qpair * (kTilesPerCta * kTileRows);
+    const int ntiles = (q0 + kTileRows < p.N) ? 2 : 1;
+    const int nkb = p.n_kblocks;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (threadIdx.x == 0) {
+        for (int t = 0; t < 2; ++t) ptx::mbar_init(bar(kBarQFull + t), 1);
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(bar(kBarKvFull + s), 1);
+            ptx::mbar_init(bar(kBarKvEmpty + s), 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            ptx::mbar_init(bar(kBarSFull + t), 1);
+            ptx::mbar_init(bar(kBarPFull + t), 4 * 32);
+            ptx::mbar_init(bar(kBarOFull + t), 1);
+        }
+        ptx::mbar_init(bar(kBarDrain), 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == kLoadWarp) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_holder), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp == kLoadWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int m = 0; m < 3; ++m)
+                    ptx::prefetch_tensormap(&p.maps[m][width_class(chunk_width(DP, c))]);
+            for (int t = 0; t < ntiles; ++t) {
+                ptx::mbar_arrive_expect_tx(bar(kBarQFull + t), TILE);
+#pragma unroll
+                for (int c = 0; c < NCH; ++c)
+                    ptx::tma_load_4d(sQ + t * TILE + 256 * chunk_col(DP, c),
+                                     &p.maps[0][width_class(chunk_width(DP, c))], chunk_col(DP, c),
+                                     h, q0 + t * kTileRows, b, bar(kBarQFull + t));
+            }
+            int issued = 0;
+            bool ok = true;
+            for (int j = 0; j < nkb && ok; ++j) {
+                for (int kv = 0; kv < 2; ++kv) {
+                    const int idx = 2 * j + kv;
+                    const int slot = idx % kStages;
+                    const uint32_t phase = (uint32_t)(idx / kStages) & 1u;
+                    if (!wait_one(bar(kBarKvEmpty + slot), phase ^ 1u, abort_flag, tmo, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    if (kv == 1 && j == 0 && (p.flags & kFlagSkipFirstVLoad)) {
+                        issued = idx + 1;
+                        continue;  // test-only: never fill this slot
+                    }
+                    ptx::mbar_arrive_expect_tx(bar(kBarKvFull + slot), TILE);
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c)
+                        ptx::tma_load_4d(sKV + slot * TILE + 256 * chunk_col(DP, c),
+                                         &p.maps[1 + kv][width_class(chunk_width(DP, c))],
+                                         chunk_col(DP, c), h, j * kBlockKeys, b,
+                                         bar(kBarKvFull + slot));
+                    issued = idx + 1;
+                }
+            }
+            if (*abort_flag) {
+                // let every copy this CTA started land before the CTA exits
+                const uint64_t drain_ns = 200000000ull;
+                for (int t = 0; t < ntiles; ++t) wait_drain(bar(kBarQFull + t), 0, drain_ns);
+                for (int idx = issued - 1; idx >= 0 && idx >= issued - kStages; --idx) {
+                    if ((p.flags & kFlagSkipFirstVLoad) && idx == 1) continue;
+                    wait_drain(bar(kBarKvFull + idx % kStages), (uint32_t)(idx / kStages) & 1u,
+                               drain_ns);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_f16(kBF16, kBlockKeys, false);
+            auto issue_s = [&](int t, int slot) {
+                const uint32_t d = tmem + (uint32_t)(t * 128);
+                int step = 0;
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+                    const int w = chunk_width(DP, c);
+                    const uint32_t qa = sQ + t * TILE + 256 * chunk_col(DP, c);
+                    const uint32_t kb = sKV + slot * TILE + 256 * chunk_col(DP, c);
+                    const uint32_t sbo = 16u * (uint32_t)w;
+#pragma unroll
+                    for (int kk = 0; kk < w / 16; ++kk) {
+                        ptx::mma_ss(d, sdesc(qa + 32 * kk, 16, sbo, swizzle_code(w)),
+                                    sdesc(kb + 32 * kk, 16, sbo, swizzle_code(w)), idS,
+                                    step > 0 ? 1u : 0u);
+                        ++step;
+                    }
+                }
+            };
+            auto issue_pv = [&](int t, int slot, bool accumulate) {
+                const uint32_t d = tmem + 256u + (uint32_t)(t * 128);
+                const uint32_t a = tmem + (uint32_t)(t * 128);
+#pragma unroll
+                for (int ks = 0; ks < kBlockKeys / 16; ++ks) {
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c) {
+                        const int w = chunk_width(DP, c);
+                        const uint32_t vb = sKV + slot * TILE + 256 * chunk_col(DP, c) + ks * 32 * w;
+                        ptx::mma_ts(d + (uint32_t)chunk_col(DP, c), a + (uint32_t)(ks * 8),
+                                    sdesc(vb, 256u * (uint32_t)w, 16u * (uint32_t)w, swizzle_code(w)),
+                                    idesc_f16(kBF16, w, true), (accumulate || ks > 0) ? 1u : 0u);
+                    }
+                }
+            };
+
+            bool ok = true;
+            for (int t = 0; t < ntiles && ok; ++t) ok = wait_one(bar(kBarQFull + t), 0, abort_flag, tmo, 2);
+            if (ok) ok = wait_one(bar(kBarKvFull + 0), 0, abort_flag, tmo, 3);
+            if (ok) {
+                ptx::tc_fence_after();
+                for (int t = 0; t < ntiles; ++t) {
+                    issue_s(t, 0);
+                    ptx::mma_commit(bar(kBarSFull + t));
+                }
+                ptx::mma_commit(bar(kBarKvEmpty + 0));
+            }
+            for (int j = 0; j < nkb && ok; ++j) {
+                const int vidx = 2 * j + 1, vslot = vidx % kStages;
+                const int kidx = 2 * j + 2, kslot = kidx % kStages;
+                if (!wait_one(bar(kBarKvFull + vslot), (uint32_t)(vidx / kStages) & 1u, abort_flag, tmo, 4)) {
+                    ok = false;
+                    break;
+                }
+                for (int t = 0; t < ntiles; ++t) {
+                    if (!wait_one(bar(kBarPFull + t), (uint32_t)j & 1u, abort_flag, tmo, 5)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    issue_pv(t, vslot, j > 0);
+                    if (j + 1 < nkb) {
+                        if (t == 0) {
+                            if (!wait_one(bar(kBarKvFull + kslot), (uint32_t)(kidx / kStages) & 1u,
+                                          abort_flag, tmo, 6)) {
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after();
+                        }
+                        issue_s(t, kslot);
+                        ptx::mma_commit(bar(kBarSFull + t));
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit(bar(kBarKvEmpty + vslot));
+                if (j + 1 < nkb) ptx::mma_commit(bar(kBarKvEmpty + kslot));
+            }
+            if (ok) {
+                for (int t = 0; t < ntiles; ++t) ptx::mma_commit(bar(kBarOFull + t));
+            } else {
+                // every MMA issued so far must finish before TMEM is freed
+                ptx::mma_commit(bar(kBarDrain));
+                wait_drain(bar(kBarDrain), 0, 200000000ull);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int t = warp >> 2;
+        const int wq = warp & 3;
+        if (t < ntiles) {
+            const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+            const uint32_t tS = tmem + lane_base + (uint32_t)(t * 128);
+            const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(t * 128);
+            const int row = q0 + t * kTileRows + wq * 32 + lane;
+            const float c2 = p.scale_log2;
+            const bool neg = c2 < 0.f;
+            float m_used = -INFINITY;
+            float l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < nkb; ++j) {
+                if (!wait_warp(bar(kBarSFull + t), (uint32_t)j & 1u, abort_flag, tmo, 7)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                float s[kBlockKeys];
+                {
+                    uint32_t r[4][32];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tS + 32 * q, r[q]);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) s[32 * q + i] = __uint_as_float(r[q][i]);
+                }
+                const int valid = min(kBlockKeys, p.N - j * kBlockKeys);
+                const bool partial = valid < kBlockKeys;
+                const float ext = partial ? row_extreme<true>(s, valid, neg)
+                                          : row_extreme<false>(s, valid, neg);
+                const float m_blk = ext * c2;
+                const float m_new = fmaxf(m_used, m_blk);
+                const bool need = (m_new - m_used) > kRescaleThreshold;
+                float alpha = 1.f;
+                if (need) {
+                    alpha = ptx::ex2(m_used - m_new);
+                    m_used = m_new;
+                    l *= alpha;
+                }
+                if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o<DP>(tO, alpha);
+                uint32_t pk[kBlockKeys / 2];
+                l += partial ? exp_and_pack<true, kBF16>(s, valid, c2, -m_used, pk)
+                             : exp_and_pack<false, kBF16>(s, valid, c2, -m_used, pk);
+                {
+                    uint32_t w0[32], w1[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        w0[i] = pk[i];
+                        w1[i] = pk[32 + i];
+                    }
+                    ptx::tmem_st32(tS, w0);
+                    ptx::tmem_st32(tS + 32, w1);
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(bar(kBarPFull + t));
+            }
+            if (ok) ok = wait_warp(bar(kBarOFull + t), 0, abort_flag, tmo, 8);
+            if (ok) {
+                ptx::tc_fence_after();
+                uint8_t* orow = reinterpret_cast<uint8_t*>(p.out) +
+                                ((((size_t)b * p.N + (size_t)min(row, p.N - 1)) * p.H + h) * p.D) * 2;
+                store_row<DP, kBF16>(tO, 1.f / l, orow, row < p.N, p.D);
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == kLoadWarp) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace vitattn

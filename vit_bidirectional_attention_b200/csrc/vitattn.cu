@@ -1,0 +1,296 @@
+// vitattn.cu -- host side of libvitattn: argument checks, TMA tensor-map
+// encoding, kernel dispatch by padded head dimension and dtype, and the
+// extern "C" entry points declared in include/vitattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "vitattn.h"
+
+#include "fwd_kernel.cuh"
+
+namespace {
+
+using vitattn::FwdParams;
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s per in-kernel wait
+
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+    t_last_cuda_error = (int)e;
+    return VITATTN_ERR_CUDA;
+}
+
+bool overlaps(const void* a, const void* b, uint64_t bytes) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bytes && y < x + bytes;
+}
+
+int check_args(const void* q, const void* k, const void* v, const void* out, int64_t B, int64_t N,
+               int64_t H, int64_t D, float scale, int dtype) {
+    if (!q || !k || !v || !out) return VITATTN_ERR_NULL;
+    if (B < 1 || N < 1 || H < 1 || D < 1) return VITATTN_ERR_DIM;
+    if (D < 16 || D > 128 || D % 8 != 0) return VITATTN_ERR_HEADDIM;
+    if (dtype != VITATTN_BF16 && dtype != VITATTN_F16) return VITATTN_ERR_DTYPE;
+    if (!std::isfinite(scale)) return VITATTN_ERR_SCALE;
+    // sizes: TMA coordinates are int32, the per-batch stride must stay below 2^40 bytes,
+    // and the grid is one CTA per (b, h, 256 query rows)
+    if (N > (int64_t)INT32_MAX - 512 || H > (int64_t)INT32_MAX || B > (int64_t)INT32_MAX)
+        return VITATTN_ERR_DIM;
+    const uint64_t batch_stride = (uint64_t)N * (uint64_t)H * (uint64_t)D * 2u;
+    if (batch_stride >= (1ull << 40)) return VITATTN_ERR_DIM;
+    if ((uint64_t)B > (1ull << 62) / batch_stride) return VITATTN_ERR_DIM;
+    const uint64_t work = (uint64_t)B * (uint64_t)H * (uint64_t)((N + 255) / 256);
+    if (work > (uint64_t)INT32_MAX) return VITATTN_ERR_DIM;
+    const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                           reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out)) & 15u;
+    if (mis) return VITATTN_ERR_ALIGN;
+    const uint64_t bytes = batch_stride * (uint64_t)B;
+    if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
+        return VITATTN_ERR_ALIAS;
+    return VITATTN_OK;
+}
+
+// ---------------------------------------------------------------- driver entry point
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// Token-major [B, N, H, D] seen by TMA as 4-D {D, H, N, B} (innermost first);
+// one box is `width` head-dim columns x 1 head x 128 tokens x 1 batch.
+bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t N, int64_t H,
+                int64_t D, int width) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)(D * 2), (cuuint64_t)(H * D * 2),
+                                   (cuuint64_t)(N * H * D * 2)};
+    const cuuint32_t box[4] = {(cuuint32_t)width, 1u, (cuuint32_t)vitattn::kTileRows, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUtensorMapSwizzle sw = width == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : width == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+    const CUtensorMapDataType dt =
+        dtype == VITATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = fn(m, dt, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- dispatch
+
+using KernelFn = void (*)(FwdParams);
+
+template <int DP, bool BF>
+KernelFn kernel_of() {
+    return vitattn::fwd_kernel<DP, BF>;
+}
+
+KernelFn pick_kernel(int dp, int dtype) {
+    const bool bf = dtype == VITATTN_BF16;
+    switch (dp) {
+        case 16: return bf ? kernel_of<16, true>() : kernel_of<16, false>();
+        case 32: return bf ? kernel_of<32, true>() : kernel_of<32, false>();
+        case 48: return bf ? kernel_of<48, true>() : kernel_of<48, false>();
+        case 64: return bf ? kernel_of<64, true>() : kernel_of<64, false>();
+        case 80: return bf ? kernel_of<80, true>() : kernel_of<80, false>();
+        case 96: return bf ? kernel_of<96, true>() : kernel_of<96, false>();
+        case 112: return bf ? kernel_of<112, true>() : kernel_of<112, false>();
+        case 128: return bf ? kernel_of<128, true>() : kernel_of<128, false>();
+        default: return nullptr;
+    }
+}
+
+// Per device: architecture verified once; per kernel instantiation: the
+// dynamic shared-memory limit raised once.
+struct DeviceState {
+    bool checked = false;
+    bool is_sm100 = false;
+    bool smem_set[9][2] = {};
+};
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+int prepare_device(int dp, int dtype, KernelFn fn) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return VITATTN_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& st = g_dev[dev];
+    if (!st.checked) {
+        int major = 0, minor = 0;
+        e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        st.is_sm100 = (major == 10 && minor == 0);
+        st.checked = true;
+    }
+    if (!st.is_sm100) return VITATTN_ERR_DEVICE;
+    bool& done = st.smem_set[dp / 16][dtype];
+    if (!done) {
+        e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 vitattn::smem_bytes(dp));
+        if (e != cudaSuccess) return cuda_fail(e);
+        done = true;
+    }
+    return VITATTN_OK;
+}
+
+int launch(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
+           int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags) {
+    int rc = check_args(q, k, v, out, B, N, H, D, scale, dtype);
+    if (rc) return rc;
+    const int dp = (int)((D + 15) / 16 * 16);
+    KernelFn fn = pick_kernel(dp, dtype);
+    if (!fn) return VITATTN_ERR_HEADDIM;
+    rc = prepare_device(dp, dtype, fn);
+    if (rc) return rc;
+
+    FwdParams prm;
+    std::memset(&prm, 0, sizeof prm);
+    const void* src[3] = {q, k, v};
+    const int nch = vitattn::chunk_count(dp);
+    for (int c = 0; c < nch; ++c) {
+        const int w = vitattn::chunk_width(dp, c);
+        for (int m = 0; m < 3; ++m) {
+            CUtensorMap* map = &prm.maps[m][vitattn::width_class(w)];
+            if (!encode_map(map, src[m], dtype, B, N, H, D, w)) return cuda_fail(cudaErrorInvalidValue);
+        }
+    }
+    prm.out = out;
+    prm.B = (int)B;
+    prm.N = (int)N;
+    prm.H = (int)H;
+    prm.D = (int)D;
+    prm.n_qpairs = (int)((N + 255) / 256);
+    prm.n_kblocks = (int)((N + 127) / 128);
+    prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    prm.flags = flags;
+    prm.timeout_ns = kWaitTimeoutNs;
+
+    const unsigned grid = (unsigned)((uint64_t)B * (uint64_t)H * (uint64_t)prm.n_qpairs);
+    void* args[1] = {&prm};
+    cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid),
+                                     dim3(vitattn::kThreads), args,
+                                     (size_t)vitattn::smem_bytes(dp), stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return VITATTN_OK;
+}
+
+int forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
+                    int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags) {
+    int rc = check_args(q, k, v, out, B, N, H, D, scale, dtype);
+    if (rc) return rc;
+    const unsigned zero = 0;
+    cudaError_t e = cudaMemcpyToSymbolAsync(g_vitattn_status, &zero, sizeof zero, 0,
+                                            cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    rc = launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags);
+    if (rc) return rc;
+    e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned status = 0;
+    e = cudaMemcpyFromSymbol(&status, g_vitattn_status, sizeof status);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return status ? VITATTN_ERR_TIMEOUT : VITATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int vitattn_forward(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
+                    int64_t H, int64_t D, float scale, int dtype, vitattn_stream_t stream) {
+    return launch(q, k, v, out, B, N, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), 0);
+}
+
+int vitattn_forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B,
+                            int64_t N, int64_t H, int64_t D, float scale, int dtype,
+                            vitattn_stream_t stream) {
+    return forward_checked(q, k, v, out, B, N, H, D, scale, dtype,
+                           reinterpret_cast<cudaStream_t>(stream), 0);
+}
+
+// Test hook, deliberately absent from the public header: the checked entry
+// with kernel test flags (bit 0: the producer withholds the first V block so
+// that a bounded wait runs out and the timeout path is exercised).
+VITATTN_API int vitattn_test_forward_flags(const void* q, const void* k, const void* v, void* out, int64_t B,
+                               int64_t N, int64_t H, int64_t D, float scale, int dtype,
+                               vitattn_stream_t stream, int flags) {
+    return forward_checked(q, k, v, out, B, N, H, D, scale, dtype,
+                           reinterpret_cast<cudaStream_t>(stream), flags);
+}
+
+int vitattn_forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq,
+                         void* dk, void* dv, void* dout, int64_t B, int64_t N, int64_t H,
+                         int64_t D, float scale, int dtype, vitattn_stream_t stream) {
+    if (!hq || !hk || !hv || !hout) return VITATTN_ERR_NULL;
+    int rc = check_args(dq, dk, dv, dout, B, N, H, D, scale, dtype);
+    if (rc) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t bytes = (size_t)B * (size_t)N * (size_t)H * (size_t)D * 2u;
+    const void* hsrc[3] = {hq, hk, hv};
+    void* ddst[3] = {dq, dk, dv};
+    for (int i = 0; i < 3; ++i) {
+        cudaError_t e = cudaMemcpyAsync(ddst[i], hsrc[i], bytes, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    rc = launch(dq, dk, dv, dout, B, N, H, D, scale, dtype, s, 0);
+    if (rc) return rc;
+    cudaError_t e = cudaMemcpyAsync(hout, dout, bytes, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return VITATTN_OK;
+}
+
+int vitattn_check_args(const void* q, const void* k, const void* v, const void* out, int64_t B,
+                       int64_t N, int64_t H, int64_t D, float scale, int dtype) {
+    return check_args(q, k, v, out, B, N, H, D, scale, dtype);
+}
+
+const char* vitattn_strerror(int status) {
+    switch (status) {
+        case VITATTN_OK: return "ok";
+        case VITATTN_ERR_NULL: return "a required pointer is NULL";
+        case VITATTN_ERR_DIM: return "B, N, H must be >= 1 and the sizes must not overflow";
+        case VITATTN_ERR_HEADDIM: return "unsupported head dimension (need 16 <= D <= 128, D % 8 == 0)";
+        case VITATTN_ERR_DTYPE: return "dtype must be VITATTN_BF16 or VITATTN_F16";
+        case VITATTN_ERR_ALIGN: return "tensor pointers must be 16-byte aligned";
+        case VITATTN_ERR_ALIAS: return "out overlaps q, k or v";
+        case VITATTN_ERR_CUDA: return "CUDA error (see vitattn_last_cuda_error)";
+        case VITATTN_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
+        case VITATTN_ERR_SCALE: return "scale must be finite";
+        case VITATTN_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+        default: return "unknown status";
+    }
+}
+
+int vitattn_last_cuda_error(void) { return t_last_cuda_error; }
+
+int vitattn_version(void) { return kVersion; }
+
+int vitattn_launches_per_call(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,146 @@
+"""Thin ctypes binding of libvitattn (the C ABI in ``include/vitattn.h``).
+
+Argument marshalling only: every step of the attention runs in the CUDA
+library.  There is no fallback: if ``libvitattn.so`` is missing this module
+raises on first use, and a failing call raises :class:`VitAttnError`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvitattn.so")
+
+BF16, F16 = 0, 1
+
+STATUS_NAMES = {
+    0: "VITATTN_OK",
+    -1: "VITATTN_ERR_NULL",
+    -2: "VITATTN_ERR_DIM",
+    -3: "VITATTN_ERR_HEADDIM",
+    -4: "VITATTN_ERR_DTYPE",
+    -5: "VITATTN_ERR_ALIGN",
+    -6: "VITATTN_ERR_ALIAS",
+    -7: "VITATTN_ERR_CUDA",
+    -8: "VITATTN_ERR_TIMEOUT",
+    -9: "VITATTN_ERR_SCALE",
+    -10: "VITATTN_ERR_DEVICE",
+}
+
+_lib = None
+
+
+class VitAttnError(RuntimeError):
+    def __init__(self, status: int, what: str = "vitattn"):
+        self.status = status
+        msg = f"{what}: {STATUS_NAMES.get(status, status)} ({strerror(status)})"
+        if status == -7:
+            msg += f", cudaError {lib().vitattn_last_cuda_error()}"
+        super().__init__(msg)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libvitattn.so is not built ({LIB_PATH}); "
+                              "run __graft_entry__.build() or vit_bidirectional_attention_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i64, f32, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+        fwd = [p, p, p, p, i64, i64, i64, i64, f32, i32, p]
+        L.vitattn_forward.argtypes = fwd
+        L.vitattn_forward_checked.argtypes = fwd
+        L.vitattn_test_forward_flags.argtypes = fwd + [i32]
+        L.vitattn_forward_host.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, f32, i32, p]
+        L.vitattn_check_args.argtypes = [p, p, p, p, i64, i64, i64, i64, f32, i32]
+        L.vitattn_strerror.argtypes = [i32]
+        L.vitattn_strerror.restype = ctypes.c_char_p
+        for f in (L.vitattn_forward, L.vitattn_forward_checked, L.vitattn_test_forward_flags,
+                  L.vitattn_forward_host, L.vitattn_check_args, L.vitattn_last_cuda_error,
+                  L.vitattn_version, L.vitattn_launches_per_call):
+            f.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return lib().vitattn_strerror(int(status)).decode()
+
+
+def version() -> int:
+    return int(lib().vitattn_version())
+
+
+def launches_per_call() -> int:
+    return int(lib().vitattn_launches_per_call())
+
+
+def check_args(q, k, v, out, B, N, H, D, scale, dtype) -> int:
+    """Status the library's argument checks give (pointers as ints); no CUDA call."""
+    return int(lib().vitattn_check_args(q, k, v, out, B, N, H, D, float(scale), dtype))
+
+
+def forward_ptr(q, k, v, out, B, N, H, D, scale, dtype, stream=0, checked=False, flags=0) -> int:
+    """Raw call on device pointers (ints); returns the status code."""
+    L = lib()
+    args = (q, k, v, out, B, N, H, D, float(scale), dtype, stream)
+    if flags:
+        return int(L.vitattn_test_forward_flags(*args, int(flags)))
+    if checked:
+        return int(L.vitattn_forward_checked(*args))
+    return int(L.vitattn_forward(*args))
+
+
+def forward_host_ptr(hq, hk, hv, hout, dq, dk, dv, dout, B, N, H, D, scale, dtype, stream=0) -> int:
+    """Raw host-buffer call (copies in, kernel, copy out, all enqueued on stream)."""
+    return int(lib().vitattn_forward_host(hq, hk, hv, hout, dq, dk, dv, dout, B, N, H, D,
+                                          float(scale), dtype, stream))
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float16:
+        return F16
+    raise TypeError(f"vitattn supports bfloat16 and float16 tensors, got {t.dtype}")
+
+
+def forward(q, k, v, out=None, scale=None, stream=None, checked=False):
+    """O = softmax(scale * Q K^T) V per (batch, head) on CUDA tensors.
+
+    q, k, v: contiguous ``[B, N, H, D]`` bf16 / f16 CUDA tensors (token-major,
+    as a QKV linear produces them).  ``scale`` defaults to 1/sqrt(D).  Returns
+    ``out`` (allocated with torch if not given).  ``checked`` synchronises and
+    reports in-kernel timeouts.
+    """
+    import torch
+
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, N, H, D] shape")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous [B, N, H, D]")
+    dtype = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor like q")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    with torch.cuda.device(q.device):
+        rc = forward_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, D,
+                         scale, dtype, handle, checked=checked)
+    if rc != 0:
+        raise VitAttnError(rc, "vitattn_forward")
+    return out
