@@ -12,7 +12,9 @@
 //
 // with the running row maximum m_t, the row sum l_t and the rescaling of O_t
 // kept exact in the online-softmax sense: O and l are always relative to the
-// same (possibly stale) maximum, so the result is O/l at the end.  This is the
+// same (possibly stale) maximum, so the result is O/l at the end.  l_t sums the
+// probabilities after their rounding to the input dtype, i.e. the weights the
+// P.V product really uses.  This is the
 // online-softmax GEMM pair of inferencelayer "src/vision_gpu.rs" (doc of
 // `vis_attn_coop_src`: "The obstacle, and the way round it"), except that the
 // running output lives in tensor memory instead of being spilled to shared
@@ -212,7 +214,11 @@ __device__ __forceinline__ float row_extreme(const float (&s)[kBlockKeys], int v
     return fminf(a, b2);
 }
 
-// p = 2^(c*s - m) for the block, packed to 16-bit pairs; returns sum of p (f32).
+// p = 2^(c*s - m) for the block, rounded and packed to 16-bit pairs.  Returns
+// the f32 sum of the ROUNDED p: the tensor core multiplies V by exactly these
+// weights, so normalising by their own sum keeps O a true weighted average of
+// V rows (a single dominant key then gives its V row exactly, whatever the
+// rounding of its weight).
 template <bool kPartial, bool kBF16>
 __device__ __forceinline__ float exp_and_pack(const float (&s)[kBlockKeys], int valid, float c2,
                                               float neg_m, uint32_t (&pk)[kBlockKeys / 2]) {
@@ -225,9 +231,8 @@ __device__ __forceinline__ float exp_and_pack(const float (&s)[kBlockKeys], int 
             p0 = c < valid ? p0 : 0.f;
             p1 = c + 1 < valid ? p1 : 0.f;
         }
-        l0 += p0;
-        l1 += p1;
         pk[c / 2] = ptx::pack2<kBF16>(p0, p1);
+        ptx::add_halves<kBF16>(pk[c / 2], l0, l1);
     }
     return l0 + l1;
 }
