@@ -50,7 +50,8 @@ KERNEL_SOURCES = ["vit_bidirectional_attention_b200/csrc/fwd_kernel.cuh",
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for about 2 s of timed work)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -124,18 +125,28 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        import datetime
+
         rows = []
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 10:
                 continue
             try:
-                rows.append({"sm": float(parts[2]), "max": float(parts[3]), "reasons": parts[5:10]})
+                ts = datetime.datetime.strptime(parts[1], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append({"t": ts, "sm": float(parts[2]), "max": float(parts[3]),
+                             "reasons": parts[5:10]})
             except ValueError:
                 continue
-        if not rows:
+        window = "timed region"
+        inside = [r for r in rows if self.t_start is not None and self.t_start <= r["t"] <= self.t_stop]
+        if not inside:
+            # timed region shorter than the sampling period: the samples
+            # around it (warm-up and timed steps back to back) stand in
+            inside, window = rows, "warm-up + timed region"
+        if not inside:
             return None
-        loaded = [r for r in rows if r["sm"] > 0.5 * r["max"]] or rows
+        loaded = inside
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         active = set()
         for r in loaded:
@@ -144,7 +155,7 @@ class ClockSampler:
                     active.add(n)
         return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
                 "sm_max_mhz": max(r["max"] for r in loaded),
-                "reasons": sorted(active), "samples": len(loaded)}
+                "reasons": sorted(active), "samples": len(loaded), "window": window}
 
 
 def cpu_baseline(w, q, k, v, seconds: float):
@@ -153,15 +164,15 @@ def cpu_baseline(w, q, k, v, seconds: float):
 
     flops_per_row = 4.0 * w.N * w.D
     total_rows = w.B * w.N * w.H
-    rows = synth.sample_rows(w, min(64, total_rows), seed=w.seed + 11)
-    t0 = time.perf_counter()
-    oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
-    t_probe = max(time.perf_counter() - t0, 1e-6)
-    want = int(min(total_rows, max(64, len(rows) * seconds / t_probe)))
-    rows = synth.sample_rows(w, want, seed=w.seed + 13)
-    t0 = time.perf_counter()
-    oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
-    dt = time.perf_counter() - t0
+    n = min(64, total_rows)
+    for attempt in range(6):
+        rows = synth.sample_rows(w, n, seed=w.seed + 11 + attempt)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * seconds or len(rows) >= total_rows:
+            break
+        n = int(min(total_rows, max(2 * n, len(rows) * seconds / max(dt, 1e-6))))
     return {"value": flops_per_row * len(rows) / dt / 1e12, "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{len(rows)} of {total_rows} output rows (seeded), fp64, "
@@ -215,6 +226,8 @@ def run_reference(args):
 
     w = synth.WORKLOADS[args.workload]
     q, k, v = synth.make_qkv(w)
+    if args.steps is None:
+        args.steps = 5
     total_rows = w.B * w.N * w.H
     per_step = max(1.0, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
     rows_probe = synth.sample_rows(w, min(64, total_rows), seed=w.seed + 17)
@@ -289,10 +302,28 @@ def main():
 
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     sampler.start()
+    t_w = time.perf_counter()
+    warm_done = 0
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
+        while warm_done < args.warmup or time.perf_counter() - t_w < 1.0:
             step()
+            warm_done += 1
+            if warm_done % 16 == 0:
+                stream.synchronize()
     stream.synchronize()
+    if args.steps is None:
+        w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0.record(stream)
+        for _ in range(5):
+            step()
+        w1.record(stream)
+        w1.synchronize()
+        est_ms = max(w0.elapsed_time(w1) / 5, 1e-3)
+        steps = int(max(20, min(20000, 2000.0 / est_ms)))
+        steps = int(max_over_ranks(float(steps), world))
+    else:
+        steps = args.steps
+    args.steps = steps
     barrier(world)
     torch.cuda.synchronize(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -357,7 +388,7 @@ def main():
             "unit": "TFLOP/s",
             "n_gpus": world,
             "steps": args.steps,
-            "warmup": args.warmup,
+            "warmup": warm_done,
             "ms_per_step": ms_step,
             "higher_is_better": True,
             "scaling": "weak",

@@ -145,10 +145,9 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned s
     atomicCAS(&g_vitattn_status, 0u, kStatusTimeoutBase + site);
 }
 
-// One thread waits for the phase of `parity`; false on abort or timeout.
-__device__ __noinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                      uint64_t timeout_ns, unsigned site) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+// Slow path of wait_one: spin with a time limit.
+__device__ __noinline__ bool wait_one_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           uint64_t timeout_ns, unsigned site) {
     const uint64_t t0 = ptx::globaltimer_ns();
     while (true) {
         if (ptx::mbar_try_wait(bar, parity)) return true;
@@ -160,6 +159,13 @@ __device__ __noinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile in
     }
 }
 
+// One thread waits for the phase of `parity`; false on abort or timeout.
+__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         uint64_t timeout_ns, unsigned site) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    return wait_one_slow(bar, parity, abort_flag, timeout_ns, site);
+}
+
 // Wait that ignores the abort flag, for draining in-flight work before exit.
 __device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
     const uint64_t t0 = ptx::globaltimer_ns();
@@ -169,11 +175,10 @@ __device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t 
     return true;
 }
 
-// A whole warp waits; the outcome is uniform across the warp.
-__device__ __noinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       uint64_t timeout_ns, unsigned site) {
-    bool done = ptx::mbar_try_wait(bar, parity);
-    if (__all_sync(0xffffffffu, done)) return true;
+// Slow path of wait_warp (whole warp, uniform outcome).
+__device__ __noinline__ bool wait_warp_slow(uint32_t bar, uint32_t parity, bool done,
+                                            volatile int* abort_flag, uint64_t timeout_ns,
+                                            unsigned site) {
     const uint64_t t0 = ptx::globaltimer_ns();
     while (true) {
         if (!done) done = ptx::mbar_try_wait(bar, parity);
@@ -191,50 +196,87 @@ __device__ __noinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile i
     }
 }
 
+// A whole warp waits; the outcome is uniform across the warp.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t timeout_ns, unsigned site) {
+    const bool done = ptx::mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    return wait_warp_slow(bar, parity, done, abort_flag, timeout_ns, site);
+}
+
 // ---------------------------------------------------------------- softmax pieces
+
+// Extreme of N values with 3-input min/max in a tree (compile-time shape, so
+// every index is a constant and nothing leaves registers).
+template <int N, bool kNeg>
+__device__ __forceinline__ float tree3(const float* v) {
+    if constexpr (N == 1) {
+        return v[0];
+    } else if constexpr (N == 2) {
+        return kNeg ? fminf(v[0], v[1]) : fmaxf(v[0], v[1]);
+    } else {
+        constexpr int M = (N + 2) / 3;
+        float t[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const float a = v[3 * i];
+            const float b = 3 * i + 1 < N ? v[3 * i + 1] : a;
+            const float c = 3 * i + 2 < N ? v[3 * i + 2] : a;
+            t[i] = kNeg ? ptx::fmin3(a, b, c) : ptx::fmax3(a, b, c);
+        }
+        return tree3<M, kNeg>(t);
+    }
+}
 
 // Row extreme of the raw scores in the direction that maximises c * s:
 // max for c >= 0, min for c < 0.  Masked columns (>= valid) are skipped.
-template <bool kPartial>
-__device__ __forceinline__ float row_extreme(const float (&s)[kBlockKeys], int valid, bool neg) {
-    float a = neg ? INFINITY : -INFINITY, b2 = a;
-    if (!neg) {
+// Reduced 32 columns at a time so that few temporaries are live at once.
+template <bool kPartial, bool kNeg>
+__device__ __forceinline__ float row_extreme(const float (&s)[kBlockKeys], int valid) {
+    const float fill = kNeg ? INFINITY : -INFINITY;
+    float part[kBlockKeys / 32];
 #pragma unroll
-        for (int c = 0; c < kBlockKeys; c += 2) {
-            if (!kPartial || c < valid) a = fmaxf(a, s[c]);
-            if (!kPartial || c + 1 < valid) b2 = fmaxf(b2, s[c + 1]);
-        }
-        return fmaxf(a, b2);
-    }
+    for (int q = 0; q < kBlockKeys / 32; ++q) {
+        float t[32];
 #pragma unroll
-    for (int c = 0; c < kBlockKeys; c += 2) {
-        if (!kPartial || c < valid) a = fminf(a, s[c]);
-        if (!kPartial || c + 1 < valid) b2 = fminf(b2, s[c + 1]);
+        for (int i = 0; i < 32; ++i) t[i] = (!kPartial || 32 * q + i < valid) ? s[32 * q + i] : fill;
+        part[q] = tree3<32, kNeg>(t);
     }
-    return fminf(a, b2);
+    return tree3<kBlockKeys / 32, kNeg>(part);
 }
 
-// p = 2^(c*s - m) for the block, rounded and packed to 16-bit pairs.  Returns
-// the f32 sum of the ROUNDED p: the tensor core multiplies V by exactly these
+// p = 2^(c*s - m) for one block, rounded to the input dtype and written to
+// TMEM as 16-bit pairs at tP (64 columns), 32 scores at a time.  Returns the
+// f32 sum of the ROUNDED p: the tensor core multiplies V by exactly these
 // weights, so normalising by their own sum keeps O a true weighted average of
 // V rows (a single dominant key then gives its V row exactly, whatever the
 // rounding of its weight).
 template <bool kPartial, bool kBF16>
-__device__ __forceinline__ float exp_and_pack(const float (&s)[kBlockKeys], int valid, float c2,
-                                              float neg_m, uint32_t (&pk)[kBlockKeys / 2]) {
-    float l0 = 0.f, l1 = 0.f;
+__device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], int valid, float c2,
+                                                float neg_m, uint32_t tP) {
+    float acc[8];
 #pragma unroll
-    for (int c = 0; c < kBlockKeys; c += 2) {
-        float p0 = ptx::ex2(fmaf(s[c], c2, neg_m));
-        float p1 = ptx::ex2(fmaf(s[c + 1], c2, neg_m));
-        if (kPartial) {
-            p0 = c < valid ? p0 : 0.f;
-            p1 = c + 1 < valid ? p1 : 0.f;
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int q = 0; q < kBlockKeys / 32; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int c = 32 * q + 2 * i;
+            const float2 x = ptx::ffma2(make_float2(s[c], s[c + 1]), make_float2(c2, c2),
+                                        make_float2(neg_m, neg_m));
+            float p0 = ptx::ex2(x.x);
+            float p1 = ptx::ex2(x.y);
+            if (kPartial) {
+                p0 = c < valid ? p0 : 0.f;
+                p1 = c + 1 < valid ? p1 : 0.f;
+            }
+            pk[i] = ptx::pack2<kBF16>(p0, p1);
+            ptx::add_halves<kBF16>(pk[i], acc[2 * (i & 3)], acc[2 * (i & 3) + 1]);
         }
-        pk[c / 2] = ptx::pack2<kBF16>(p0, p1);
-        ptx::add_halves<kBF16>(pk[c / 2], l0, l1);
+        ptx::tmem_st16(tP + 16 * q, pk);
     }
-    return l0 + l1;
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
 // Multiply this thread's row of O (DP columns of TMEM at tO) by alpha.
@@ -531,8 +573,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 }
                 const int valid = min(kBlockKeys, p.N - j * kBlockKeys);
                 const bool partial = valid < kBlockKeys;
-                const float ext = partial ? row_extreme<true>(s, valid, neg)
-                                          : row_extreme<false>(s, valid, neg);
+                const float ext = partial ? (neg ? row_extreme<true, true>(s, valid)
+                                                 : row_extreme<true, false>(s, valid))
+                                          : (neg ? row_extreme<false, true>(s, valid)
+                                                 : row_extreme<false, false>(s, valid));
                 const float m_blk = ext * c2;
                 const float m_new = fmaxf(m_used, m_blk);
                 const bool need = (m_new - m_used) > kRescaleThreshold;
@@ -542,20 +586,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     m_used = m_new;
                     l *= alpha;
                 }
+                l += partial ? exp_pack_store<true, kBF16>(s, valid, c2, -m_used, tS)
+                             : exp_pack_store<false, kBF16>(s, valid, c2, -m_used, tS);
+                // O_t holds P.V up to block j-1 (complete: the S_t,j commit came after
+                // it); bring it to the new reference maximum before P_t,j.V_j is issued.
                 if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o<DP>(tO, alpha);
-                uint32_t pk[kBlockKeys / 2];
-                l += partial ? exp_and_pack<true, kBF16>(s, valid, c2, -m_used, pk)
-                             : exp_and_pack<false, kBF16>(s, valid, c2, -m_used, pk);
-                {
-                    uint32_t w0[32], w1[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        w0[i] = pk[i];
-                        w1[i] = pk[32 + i];
-                    }
-                    ptx::tmem_st32(tS, w0);
-                    ptx::tmem_st32(tS + 32, w1);
-                }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(bar(kBarPFull + t));
