@@ -36,7 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from vit_bidirectional_attention_b200 import synth  # noqa: E402
+from vit_bidirectional_attention_b200 import ranks, synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "batched"
 METRIC = "attention fwd TFLOP/s (4·B·H·N²·D) and % of B200 dense BF16 tensor peak"
@@ -182,38 +182,21 @@ def cpu_baseline(w, q, k, v, seconds: float):
 def dist_setup(args):
     import torch
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = ranks.env_world()
     if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        ranks.init("nccl", world, device=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
     return world, rank, local
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.barrier()
+    ranks.barrier(world)
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return ranks.max_over_ranks(x, world, device="cuda")
 
 
 def run_reference(args):
@@ -339,7 +322,7 @@ def main():
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
     clocks = sampler.stop()
     ms_step = ms_total / args.steps
-    tflops = w.flops * args.steps * world / (ms_total * 1e-3) / 1e12
+    tflops = ranks.job_throughput(w.flops, args.steps, world, ms_total)
     per_gpu_tflops = w.flops / (ms_step * 1e-3) / 1e12
 
     # end to end through the host-buffer entry point
@@ -366,7 +349,7 @@ def main():
     e1.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = w.flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = ranks.job_throughput(w.flops, e2e_steps, world, e2e_ms)
 
     peaks, peak_src = measured_peaks()
     if peaks:
@@ -425,11 +408,7 @@ def main():
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.finish(world)
     if result is not None:
         print(json.dumps(result), flush=True)
     return 0

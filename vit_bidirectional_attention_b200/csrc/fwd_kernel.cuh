@@ -245,6 +245,32 @@ __device__ __forceinline__ float row_extreme(const float (&s)[kBlockKeys], int v
     return tree3<kBlockKeys / 32, kNeg>(part);
 }
 
+// Pairs of exponentials (out of every 16 pairs) computed by the polynomial on
+// the FMA/ALU pipes instead of ex2.approx on the MUFU pipe, which runs at 16
+// results per clock per SM and is otherwise the softmax's bottleneck.
+constexpr int kPolyPairs = 0;
+__host__ __device__ constexpr bool poly_pair(int i) { return (i * kPolyPairs) % 16 < kPolyPairs; }
+
+// 2^x for a pair, on the FMA and ALU pipes.  Cody-Waite style split
+// x = j + f with j = round(x) (the 1.5 * 2^23 addition trick leaves j in the
+// low mantissa bits of t) and f in [-1/2, 1/2]; 2^f from a degree-3 minimax
+// polynomial (Remez exchange on the relative error: max 7.5e-5, below the
+// 2^-9 half-ulp of bf16 and about a sixth of an f16 ulp); j is then added to
+// the exponent field.  x is clamped below at -125 so the exponent stays normal.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    const float2 t = ptx::fadd2(x, magic);
+    const float2 f = ptx::fsub2(x, ptx::fsub2(t, magic));
+    float2 p = ptx::ffma2(f, make_float2(0.0551716685f, 0.0551716685f),
+                          make_float2(0.2426111251f, 0.2426111251f));
+    p = ptx::ffma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
+    p = ptx::ffma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // p = 2^(c*s - m) for one block, rounded to the input dtype and written to
 // TMEM as 16-bit pairs at tP (64 columns), 32 scores at a time.  Returns the
 // f32 sum of the ROUNDED p: the tensor core multiplies V by exactly these
@@ -254,9 +280,9 @@ __device__ __forceinline__ float row_extreme(const float (&s)[kBlockKeys], int v
 template <bool kPartial, bool kBF16>
 __device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], int valid, float c2,
                                                 float neg_m, uint32_t tP) {
-    float acc[8];
+    float acc[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 4; ++i) acc[i] = 0.f;
 #pragma unroll
     for (int q = 0; q < kBlockKeys / 32; ++q) {
         uint32_t pk[16];
@@ -265,18 +291,25 @@ __device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], in
             const int c = 32 * q + 2 * i;
             const float2 x = ptx::ffma2(make_float2(s[c], s[c + 1]), make_float2(c2, c2),
                                         make_float2(neg_m, neg_m));
-            float p0 = ptx::ex2(x.x);
-            float p1 = ptx::ex2(x.y);
+            float p0, p1;
+            if (poly_pair(i)) {
+                const float2 e = exp2_poly2(x);
+                p0 = e.x;
+                p1 = e.y;
+            } else {
+                p0 = ptx::ex2(x.x);
+                p1 = ptx::ex2(x.y);
+            }
             if (kPartial) {
                 p0 = c < valid ? p0 : 0.f;
                 p1 = c + 1 < valid ? p1 : 0.f;
             }
             pk[i] = ptx::pack2<kBF16>(p0, p1);
-            ptx::add_halves<kBF16>(pk[i], acc[2 * (i & 3)], acc[2 * (i & 3) + 1]);
+            ptx::add_halves<kBF16>(pk[i], acc[2 * (i & 1)], acc[2 * (i & 1) + 1]);
         }
         ptx::tmem_st16(tP + 16 * q, pk);
     }
-    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
 // Multiply this thread's row of O (DP columns of TMEM at tO) by alpha.
@@ -454,37 +487,55 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            // Descriptors are built once per chunk and phase; a K step then
+            // only adds a constant to the start-address field (16-byte units),
+            // so the single issuing thread spends its time issuing MMAs.
             constexpr uint32_t idS = idesc_f16(kBF16, kBlockKeys, false);
             auto issue_s = [&](int t, int slot) {
                 const uint32_t d = tmem + (uint32_t)(t * 128);
-                int step = 0;
 #pragma unroll
                 for (int c = 0; c < NCH; ++c) {
                     const int w = chunk_width(DP, c);
-                    const uint32_t qa = sQ + t * TILE + 256 * chunk_col(DP, c);
-                    const uint32_t kb = sKV + slot * TILE + 256 * chunk_col(DP, c);
-                    const uint32_t sbo = 16u * (uint32_t)w;
+                    const uint64_t qd = sdesc(sQ + t * TILE + 256 * chunk_col(DP, c), 16,
+                                              16u * (uint32_t)w, swizzle_code(w));
+                    const uint64_t kd = sdesc(sKV + slot * TILE + 256 * chunk_col(DP, c), 16,
+                                              16u * (uint32_t)w, swizzle_code(w));
 #pragma unroll
-                    for (int kk = 0; kk < w / 16; ++kk) {
-                        ptx::mma_ss(d, sdesc(qa + 32 * kk, 16, sbo, swizzle_code(w)),
-                                    sdesc(kb + 32 * kk, 16, sbo, swizzle_code(w)), idS,
-                                    step > 0 ? 1u : 0u);
-                        ++step;
-                    }
+                    for (int kk = 0; kk < w / 16; ++kk)
+                        ptx::mma_ss(d, qd + 2u * kk, kd + 2u * kk, idS,
+                                    (c == 0 && kk == 0) ? 0u : 1u);
                 }
             };
+            // P.V: the 64-column chunks of V form one MMA with N = 64 * n64 (the
+            // second 64-column swizzle atom sits one chunk, 16 KB, further: the
+            // leading byte offset); narrower tail chunks get an MMA each.
+            constexpr int N64 = DP / 64;
+            constexpr int NTAIL = NCH - N64;
             auto issue_pv = [&](int t, int slot, bool accumulate) {
                 const uint32_t d = tmem + 256u + (uint32_t)(t * 128);
                 const uint32_t a = tmem + (uint32_t)(t * 128);
+                const uint32_t vbase = sKV + slot * TILE;
+                const uint64_t vd64 = sdesc(vbase, 128u * 128u, 16u * 64u, swizzle_code(64));
+                uint64_t vdt[NTAIL > 0 ? NTAIL : 1];
+#pragma unroll
+                for (int i = 0; i < NTAIL; ++i) {
+                    const int c = N64 + i;
+                    const int w = chunk_width(DP, c);
+                    vdt[i] = sdesc(vbase + 256 * chunk_col(DP, c), 256u * (uint32_t)w,
+                                   16u * (uint32_t)w, swizzle_code(w));
+                }
 #pragma unroll
                 for (int ks = 0; ks < kBlockKeys / 16; ++ks) {
+                    const uint32_t acc = (accumulate || ks > 0) ? 1u : 0u;
+                    if (N64 > 0)
+                        ptx::mma_ts(d, a + (uint32_t)(ks * 8), vd64 + (uint64_t)(2 * 64 * ks),
+                                    idesc_f16(kBF16, 64 * N64, true), acc);
 #pragma unroll
-                    for (int c = 0; c < NCH; ++c) {
+                    for (int i = 0; i < NTAIL; ++i) {
+                        const int c = N64 + i;
                         const int w = chunk_width(DP, c);
-                        const uint32_t vb = sKV + slot * TILE + 256 * chunk_col(DP, c) + ks * 32 * w;
                         ptx::mma_ts(d + (uint32_t)chunk_col(DP, c), a + (uint32_t)(ks * 8),
-                                    sdesc(vb, 256u * (uint32_t)w, 16u * (uint32_t)w, swizzle_code(w)),
-                                    idesc_f16(kBF16, w, true), (accumulate || ks > 0) ? 1u : 0u);
+                                    vdt[i] + (uint64_t)(2 * w * ks), idesc_f16(kBF16, w, true), acc);
                     }
                 }
             };
