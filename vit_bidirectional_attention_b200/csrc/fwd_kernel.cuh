@@ -23,11 +23,16 @@
 // hold).  Keys past N are masked to probability 0 (same page, "Keys past the
 // span ... are masked to zero probability").
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax for query tile 0 (TMEM lanes 0..127 through warp%4)
-//   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer (one lane) and TMEM allocator (whole warp)
-//   warp  9    MMA issuer (one lane)
+// Warp roles (384 threads, three warpgroups):
+//   warps 0-3    softmax for query tile 0 (TMEM lanes 0..127 through warp%4)
+//   warps 4-7    softmax for query tile 1
+//   warp  8      TMA producer (one lane) and TMEM allocator (whole warp)
+//   warp  9      MMA issuer (one lane)
+//   warps 10-11  idle (they complete the third warpgroup)
+// Registers: the launch gives every thread kLaunchRegs; the third warpgroup
+// then gives most of its share back (setmaxnreg.dec to kSideRegs) and the two
+// softmax warpgroups take it (setmaxnreg.inc to kSoftmaxRegs), so a softmax
+// thread can hold its 128 scores and still keep many exponentials in flight.
 //
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   [  0,128)  S_0, later P_0 (16-bit pairs in the first 64 columns)
@@ -63,9 +68,17 @@ constexpr int kTileRows = 128;    // query rows per tile = TMEM lanes
 constexpr int kBlockKeys = 128;   // keys per K/V block
 constexpr int kTilesPerCta = 2;
 constexpr int kStages = 4;        // K/V ring slots (K_j, V_j, K_j+1, V_j+1)
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
+// Register split: 3 warps share each SMSP register file (16384 x 32-bit), so a
+// 384-thread block launches at 168 per thread; 2*224 + 56 = 3*168 per SMSP and
+// 256*224 + 128*56 = 384*168 per block: the reallocation never waits forever.
+constexpr uint32_t kLaunchRegs = 168;
+constexpr uint32_t kSoftmaxRegs = 224;
+constexpr uint32_t kSideRegs = 56;
+static_assert(2 * kSoftmaxRegs + kSideRegs == 3 * kLaunchRegs, "register split per SMSP");
+static_assert(256 * kSoftmaxRegs + 128 * kSideRegs == kThreads * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
 
@@ -146,7 +159,7 @@ __device__ __forceinline__ void raise_abort(volatile int* abort_flag, unsigned s
 }
 
 // Slow path of wait_one: spin with a time limit.
-__device__ __noinline__ bool wait_one_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+__device__ __forceinline__ bool wait_one_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                            uint64_t timeout_ns, unsigned site) {
     const uint64_t t0 = ptx::globaltimer_ns();
     while (true) {
@@ -167,7 +180,7 @@ __device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile
 }
 
 // Wait that ignores the abort flag, for draining in-flight work before exit.
-__device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
     const uint64_t t0 = ptx::globaltimer_ns();
     while (!ptx::mbar_try_wait(bar, parity)) {
         if (ptx::globaltimer_ns() - t0 > timeout_ns) return false;
@@ -176,7 +189,7 @@ __device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t 
 }
 
 // Slow path of wait_warp (whole warp, uniform outcome).
-__device__ __noinline__ bool wait_warp_slow(uint32_t bar, uint32_t parity, bool done,
+__device__ __forceinline__ bool wait_warp_slow(uint32_t bar, uint32_t parity, bool done,
                                             volatile int* abort_flag, uint64_t timeout_ns,
                                             unsigned site) {
     const uint64_t t0 = ptx::globaltimer_ns();
@@ -431,6 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
+    // Each role's register budget is set inside its own branch, so that the
+    // compiler allocates the softmax code against the larger budget.
+    if (warp >= kLoadWarp) {
+    ptx::setmaxnreg_dec<kSideRegs>();
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -591,7 +608,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             }
         }
         __syncwarp();
+    }
     } else {
+        ptx::setmaxnreg_inc<kSoftmaxRegs>();
         // ------------------------------------------------------------ softmax
         const int t = warp >> 2;
         const int wq = warp & 3;
