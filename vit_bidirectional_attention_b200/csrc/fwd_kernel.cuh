@@ -34,11 +34,17 @@
 // softmax warpgroups take it (setmaxnreg.inc to kSoftmaxRegs), so a softmax
 // thread can hold its 128 scores and still keep many exponentials in flight.
 //
+// Work order.  The (tile, key block) units are numbered s = ntiles*j + t.
+// Unit s gets S buffer s % NS, where NS = 3 S buffers fit in TMEM when
+// DP <= 64 and 2 otherwise.  The MMA warp issues S for the first NS units,
+// then for every unit s: O_t += P_s V_j, followed by S for unit s + NS in the
+// buffer P_s has just been read from.  With NS = 3 a tile's next S is
+// computed while its softmax still works on the current block; with NS = 2
+// this is the classic two-tile ping-pong.
+//
 // Tensor memory (512 columns x 128 lanes x 32 bit):
-//   [  0,128)  S_0, later P_0 (16-bit pairs in the first 64 columns)
-//   [128,256)  S_1 / P_1
-//   [256,384)  O_0 (DP columns used)
-//   [384,512)  O_1
+//   [128*b, 128*b+128)  S buffer b < NS, later P (16-bit pairs in its first 64 columns)
+//   [128*NS + oc*t, ...)  O_t, DP of its oc = 64 (DP <= 64) or 128 columns used
 //
 // Shared memory: Q_0, Q_1 and a ring of kStages K/V slots, each a 128 x DP
 // tile stored as column chunks of 64 / 32 / 16 elements (SW128 / SW64 / SW32
@@ -86,9 +92,15 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max g
 constexpr int kBarQFull = 0;                         // [2]
 constexpr int kBarKvFull = 2;                        // [kStages]
 constexpr int kBarKvEmpty = kBarKvFull + kStages;    // [kStages]
-constexpr int kBarSFull = kBarKvEmpty + kStages;     // [2]
-constexpr int kBarPFull = kBarSFull + 2;             // [2]
-constexpr int kBarOFull = kBarPFull + 2;             // [2]
+constexpr int kMaxSBufs = 3;
+constexpr int kBarSFull = kBarKvEmpty + kStages;     // [kMaxSBufs] one per S buffer
+// [2 tiles][2] P written (and O rescaled) for blocks of even / odd index: with
+// the S look-ahead a tile's softmax can finish block j+1 before the MMA warp
+// has consumed block j, and one barrier per tile could then run two phases
+// ahead of its waiter; block j+2 needs P.V of block j first, so two cannot.
+constexpr int kBarPFull = kBarSFull + kMaxSBufs;
+constexpr int kBarOReady = kBarPFull + 4;            // [2] per tile: a P.V product finished
+constexpr int kBarOFull = kBarOReady + 2;            // [2] per tile: the last P.V finished
 constexpr int kBarDrain = kBarOFull + 2;             // [1]
 constexpr int kNumBars = kBarDrain + 1;
 
@@ -117,6 +129,25 @@ __host__ __device__ constexpr int width_class(int w) { return w == 64 ? 0 : (w =
 __host__ __device__ constexpr uint32_t swizzle_code(int w) { return w == 64 ? 2u : (w == 32 ? 4u : 6u); }
 
 __host__ __device__ constexpr int tile_bytes(int dp) { return kTileRows * dp * 2; }
+// TMEM: kTilesPerCta O accumulators of o_cols(dp) columns at the top, and as
+// many 128-column S/P buffers below them as fit (3 when dp <= 64, else 2).
+__host__ __device__ constexpr int o_cols(int dp) { return dp <= 64 ? 64 : 128; }
+__host__ __device__ constexpr int s_buffers(int dp) {
+    return (512 - kTilesPerCta * o_cols(dp)) / kBlockKeys;
+}
+// S buffers in use.  A third buffer is only used with two query tiles: then
+// S for unit s is issued after P.V of unit s-3, so when tile t's softmax sees
+// S(t, j) the product P.V(t, j-2) has finished, which is what makes the
+// parity wait for P.V(t, j-1) in the O rescale unambiguous.  With one tile and
+// three buffers only P.V(j-3) would be known complete.
+__host__ __device__ constexpr int active_s_buffers(int ns, int ntiles) {
+    return ntiles == 2 ? ns : (ns < 2 ? ns : 2);
+}
+// With ns buffers and ntiles tiles, S(t, j) is issued after P.V of unit
+// ntiles*j + t - ns.  When that is P.V(t, j-1) itself (ns == ntiles), seeing
+// S(t, j) already proves P.V(t, j-1) done and the separate "P.V done"
+// barrier (one extra tcgen05.commit per product) is not needed.
+__host__ __device__ constexpr bool pv_done_needed(int ns, int ntiles) { return ns != ntiles; }
 __host__ __device__ constexpr int smem_bytes(int dp) {
     return (kTilesPerCta + kStages) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
 }
@@ -426,9 +457,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             ptx::mbar_init(bar(kBarKvFull + s), 1);
             ptx::mbar_init(bar(kBarKvEmpty + s), 1);
         }
+        for (int b = 0; b < kMaxSBufs; ++b) ptx::mbar_init(bar(kBarSFull + b), 1);
         for (int t = 0; t < 2; ++t) {
-            ptx::mbar_init(bar(kBarSFull + t), 1);
-            ptx::mbar_init(bar(kBarPFull + t), 4 * 32);
+            ptx::mbar_init(bar(kBarPFull + 2 * t), 4 * 32);
+            ptx::mbar_init(bar(kBarPFull + 2 * t + 1), 4 * 32);
+            ptx::mbar_init(bar(kBarOReady + t), 1);
             ptx::mbar_init(bar(kBarOFull + t), 1);
         }
         ptx::mbar_init(bar(kBarDrain), 1);
@@ -489,8 +522,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     issued = idx + 1;
                 }
             }
-            if (*abort_flag) {
-                // let every copy this CTA started land before the CTA exits
+            {
+                // let every copy this CTA started land before the CTA exits (in a
+                // normal run they all have; after an abort some may not have been
+                // waited for).  The last fill of each slot is its latest phase, so
+                // its parity is unambiguous whether or not it was consumed.
                 const uint64_t drain_ns = 200000000ull;
                 for (int t = 0; t < ntiles; ++t) wait_drain(bar(kBarQFull + t), 0, drain_ns);
                 for (int idx = issued - 1; idx >= 0 && idx >= issued - kStages; --idx) {
@@ -508,8 +544,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             // only adds a constant to the start-address field (16-byte units),
             // so the single issuing thread spends its time issuing MMAs.
             constexpr uint32_t idS = idesc_f16(kBF16, kBlockKeys, false);
-            auto issue_s = [&](int t, int slot) {
-                const uint32_t d = tmem + (uint32_t)(t * 128);
+            constexpr int NS = s_buffers(DP);
+            constexpr int OC = o_cols(DP);
+            auto mma_s = [&](int t, int slot, int buf) {
+                const uint32_t d = tmem + (uint32_t)(buf * kBlockKeys);
 #pragma unroll
                 for (int c = 0; c < NCH; ++c) {
                     const int w = chunk_width(DP, c);
@@ -528,9 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             // leading byte offset); narrower tail chunks get an MMA each.
             constexpr int N64 = DP / 64;
             constexpr int NTAIL = NCH - N64;
-            auto issue_pv = [&](int t, int slot, bool accumulate) {
-                const uint32_t d = tmem + 256u + (uint32_t)(t * 128);
-                const uint32_t a = tmem + (uint32_t)(t * 128);
+            auto mma_pv = [&](int t, int slot, int buf, bool accumulate) {
+                const uint32_t d = tmem + (uint32_t)(NS * kBlockKeys + t * OC);
+                const uint32_t a = tmem + (uint32_t)(buf * kBlockKeys);
                 const uint32_t vbase = sKV + slot * TILE;
                 const uint64_t vd64 = sdesc(vbase, 128u * 128u, 16u * 64u, swizzle_code(64));
                 uint64_t vdt[NTAIL > 0 ? NTAIL : 1];
@@ -556,48 +594,70 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     }
                 }
             };
+            // K_j and V_j occupy ring entries 2j and 2j+1 (the producer's order).
+            auto kv_slot = [](int idx) { return idx % kStages; };
+            auto kv_parity = [](int idx) { return (uint32_t)(idx / kStages) & 1u; };
+            const int T = ntiles;
+            const int total = T * nkb;
+            const int ns = active_s_buffers(NS, T);
+            const bool track_pv = pv_done_needed(ns, T);
+            // A cursor walks the units s = T*j + t in order, keeping (t, j) and the
+            // S buffer s mod ns without divisions (this thread is on the critical path).
+            struct Cursor {
+                int t, j, buf;
+            };
+            auto advance = [&](Cursor& c) {
+                if (++c.t == T) {
+                    c.t = 0;
+                    ++c.j;
+                }
+                if (++c.buf == ns) c.buf = 0;
+            };
+            // S for one unit into its buffer; K_j is waited for by its first unit
+            // and released after its last.
+            auto issue_s = [&](const Cursor& c) -> bool {
+                if (c.t == 0) {
+                    if (!wait_one(bar(kBarKvFull + kv_slot(2 * c.j)), kv_parity(2 * c.j), abort_flag, tmo, 3))
+                        return false;
+                    ptx::tc_fence_after();
+                }
+                mma_s(c.t, kv_slot(2 * c.j), c.buf);
+                ptx::mma_commit(bar(kBarSFull + c.buf));
+                if (c.t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * c.j)));
+                return true;
+            };
+            // O_t += P V_j; V_j is waited for by its first unit and released after its last.
+            auto issue_pv = [&](const Cursor& c) -> bool {
+                const int t = c.t, j = c.j;
+                if (t == 0 &&
+                    !wait_one(bar(kBarKvFull + kv_slot(2 * j + 1)), kv_parity(2 * j + 1), abort_flag, tmo, 4))
+                    return false;
+                if (!wait_one(bar(kBarPFull + 2 * t + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_flag, tmo, 5))
+                    return false;
+                ptx::tc_fence_after();
+                mma_pv(t, kv_slot(2 * j + 1), c.buf, j > 0);
+                if (track_pv) ptx::mma_commit(bar(kBarOReady + t));
+                if (t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * j + 1)));
+                return true;
+            };
 
             bool ok = true;
-            for (int t = 0; t < ntiles && ok; ++t) ok = wait_one(bar(kBarQFull + t), 0, abort_flag, tmo, 2);
-            if (ok) ok = wait_one(bar(kBarKvFull + 0), 0, abort_flag, tmo, 3);
-            if (ok) {
-                ptx::tc_fence_after();
-                for (int t = 0; t < ntiles; ++t) {
-                    issue_s(t, 0);
-                    ptx::mma_commit(bar(kBarSFull + t));
-                }
-                ptx::mma_commit(bar(kBarKvEmpty + 0));
+            for (int t = 0; t < T && ok; ++t) ok = wait_one(bar(kBarQFull + t), 0, abort_flag, tmo, 2);
+            Cursor cs{0, 0, 0};  // next unit whose S is issued
+            Cursor cp{0, 0, 0};  // next unit whose P.V is issued
+            int issued_s = 0;
+            for (; issued_s < ns && issued_s < total && ok; ++issued_s) {
+                ok = issue_s(cs);
+                advance(cs);
             }
-            for (int j = 0; j < nkb && ok; ++j) {
-                const int vidx = 2 * j + 1, vslot = vidx % kStages;
-                const int kidx = 2 * j + 2, kslot = kidx % kStages;
-                if (!wait_one(bar(kBarKvFull + vslot), (uint32_t)(vidx / kStages) & 1u, abort_flag, tmo, 4)) {
-                    ok = false;
-                    break;
+            for (int s = 0; s < total && ok; ++s) {
+                ok = issue_pv(cp);
+                advance(cp);
+                if (ok && issued_s < total) {
+                    ok = issue_s(cs);
+                    advance(cs);
+                    ++issued_s;
                 }
-                for (int t = 0; t < ntiles; ++t) {
-                    if (!wait_one(bar(kBarPFull + t), (uint32_t)j & 1u, abort_flag, tmo, 5)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::tc_fence_after();
-                    issue_pv(t, vslot, j > 0);
-                    if (j + 1 < nkb) {
-                        if (t == 0) {
-                            if (!wait_one(bar(kBarKvFull + kslot), (uint32_t)(kidx / kStages) & 1u,
-                                          abort_flag, tmo, 6)) {
-                                ok = false;
-                                break;
-                            }
-                            ptx::tc_fence_after();
-                        }
-                        issue_s(t, kslot);
-                        ptx::mma_commit(bar(kBarSFull + t));
-                    }
-                }
-                if (!ok) break;
-                ptx::mma_commit(bar(kBarKvEmpty + vslot));
-                if (j + 1 < nkb) ptx::mma_commit(bar(kBarKvEmpty + kslot));
             }
             if (ok) {
                 for (int t = 0; t < ntiles; ++t) ptx::mma_commit(bar(kBarOFull + t));
@@ -615,17 +675,29 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         const int t = warp >> 2;
         const int wq = warp & 3;
         if (t < ntiles) {
+            constexpr int NS = s_buffers(DP);
+            const int ns = active_s_buffers(NS, ntiles);
             const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-            const uint32_t tS = tmem + lane_base + (uint32_t)(t * 128);
-            const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(t * 128);
+            const uint32_t tO = tmem + lane_base + (uint32_t)(NS * kBlockKeys + t * o_cols(DP));
             const int row = q0 + t * kTileRows + wq * 32 + lane;
             const float c2 = p.scale_log2;
             const bool neg = c2 < 0.f;
             float m_used = -INFINITY;
             float l = 0.f;
             bool ok = true;
+            // unit = ntiles*j + t lives in S buffer unit % ns, as phase unit / ns of
+            // that buffer's barrier; both advance by ntiles units per block.
+            int sbuf = t % ns, sphase = t / ns;
             for (int j = 0; j < nkb; ++j) {
-                if (!wait_warp(bar(kBarSFull + t), (uint32_t)j & 1u, abort_flag, tmo, 7)) {
+                const uint32_t tS = tmem + lane_base + (uint32_t)(sbuf * kBlockKeys);
+                const uint32_t s_bar = bar(kBarSFull + sbuf);
+                const uint32_t s_par = (uint32_t)sphase & 1u;
+                sbuf += ntiles;
+                if (sbuf >= ns) {
+                    sbuf -= ns;
+                    ++sphase;
+                }
+                if (!wait_warp(s_bar, s_par, abort_flag, tmo, 7)) {
                     ok = false;
                     break;
                 }
@@ -658,12 +730,22 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 }
                 l += partial ? exp_pack_store<true, kBF16>(s, valid, c2, -m_used, tS)
                              : exp_pack_store<false, kBF16>(s, valid, c2, -m_used, tS);
-                // O_t holds P.V up to block j-1 (complete: the S_t,j commit came after
-                // it); bring it to the new reference maximum before P_t,j.V_j is issued.
-                if (j > 0 && __any_sync(0xffffffffu, need)) rescale_o<DP>(tO, alpha);
+                // Bring O_t (P.V up to block j-1) to the new reference maximum before
+                // P_t,j.V_j is issued.  The product of block j-1 may still be running:
+                // wait for it (phase j-1 of the per-tile "P.V done" barrier; the phase
+                // of block j-2 has completed by now, so the parity is unambiguous).
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    if (pv_done_needed(ns, ntiles) &&
+                        !wait_warp(bar(kBarOReady + t), (uint32_t)(j - 1) & 1u, abort_flag, tmo, 11)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    rescale_o<DP>(tO, alpha);
+                }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(bar(kBarPFull + t));
+                ptx::mbar_arrive(bar(kBarPFull + 2 * t + (j & 1)));
             }
             if (ok) ok = wait_warp(bar(kBarOFull + t), 0, abort_flag, tmo, 8);
             if (ok) {
