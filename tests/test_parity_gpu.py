@@ -40,9 +40,22 @@ def from_dev(t, dtype):
     return synth.bits_to_float32(bits, dtype).astype(np.float64)
 
 
-def run_gpu(q, k, v, scale, dtype):
+FORCE_TWO_TILES = 2
+FORCE_ONE_TILE = 4
+
+
+def run_gpu(q, k, v, scale, dtype, flags=0):
+    import torch
+
     tq, tk, tv = (to_dev(x, dtype) for x in (q, k, v))
-    out = vitattn.forward(tq, tk, tv, scale=scale, checked=True)
+    if not flags:
+        out = vitattn.forward(tq, tk, tv, scale=scale, checked=True)
+        return from_dev(out, dtype)
+    B, N, H, D = q.shape
+    out = torch.empty_like(tq)
+    rc = vitattn.forward_ptr(tq.data_ptr(), tk.data_ptr(), tv.data_ptr(), out.data_ptr(), B, N, H,
+                             D, scale, dtype, torch.cuda.current_stream().cuda_stream, flags=flags)
+    assert rc == 0, vitattn.strerror(rc)
     return from_dev(out, dtype)
 
 
@@ -94,23 +107,27 @@ def test_workload_sampled_parity_at_full_size(cuda_device, name, rows):
 SWEEP_N = [1, 2, 63, 64, 65, 127, 128, 129, 196, 255, 256, 257, 384, 912, 1024]
 
 
+@pytest.mark.parametrize("tiles", [FORCE_TWO_TILES, FORCE_ONE_TILE])
 @pytest.mark.parametrize("N", SWEEP_N)
 @pytest.mark.parametrize("D", [64, 80, 128])
-def test_sweep_tokens(cuda_device, N, D):
+def test_sweep_tokens(cuda_device, N, D, tiles):
+    """Ragged and exact token counts, with two query tiles per CTA (three S
+    buffers at D = 64) and with one."""
     q, k, v = synth.random_qkv(1, N, 2, D, synth.BF16, seed=1000 + N * 7 + D)
     scale = 1.0 / math.sqrt(D)
-    assert_close(run_gpu(q, k, v, scale, synth.BF16), oracle.attention(q, k, v, scale, synth.BF16),
-                 f"N={N} D={D}")
+    assert_close(run_gpu(q, k, v, scale, synth.BF16, flags=tiles),
+                 oracle.attention(q, k, v, scale, synth.BF16), f"N={N} D={D} tiles flag {tiles}")
 
 
+@pytest.mark.parametrize("tiles", [FORCE_TWO_TILES, FORCE_ONE_TILE])
 @pytest.mark.parametrize("dtype", [synth.BF16, synth.F16])
 @pytest.mark.parametrize("D", [16, 24, 32, 40, 48, 56, 64, 72, 80, 88, 96, 104, 112, 120, 128])
 @pytest.mark.parametrize("N", [1, 129, 257])
-def test_sweep_head_dims(cuda_device, dtype, D, N):
+def test_sweep_head_dims(cuda_device, dtype, D, N, tiles):
     q, k, v = synth.random_qkv(1, N, 3, D, dtype, seed=2000 + N * 131 + D * 3 + dtype)
     scale = 1.0 / math.sqrt(D)
-    assert_close(run_gpu(q, k, v, scale, dtype), oracle.attention(q, k, v, scale, dtype),
-                 f"N={N} D={D} dtype={dtype}")
+    assert_close(run_gpu(q, k, v, scale, dtype, flags=tiles), oracle.attention(q, k, v, scale, dtype),
+                 f"N={N} D={D} dtype={dtype} tiles flag {tiles}")
 
 
 def test_many_batches_and_heads(cuda_device):
@@ -130,6 +147,14 @@ def test_peaky_logits_rescale_path(cuda_device):
     w = synth.Workload("peaky", 1, 2048, 4, 128, synth.BF16, rank8_logit_std=4.0, index=4)
     q, k, v = synth.make_qkv(w)
     assert_close(run_gpu(q, k, v, w.scale, w.dtype), oracle.attention(q, k, v, w.scale, w.dtype))
+
+
+@pytest.mark.parametrize("tiles", [FORCE_TWO_TILES, FORCE_ONE_TILE])
+def test_peaky_rescale_with_each_tile_mode(cuda_device, tiles):
+    w = synth.Workload("peaky64", 1, 1536, 2, 64, synth.BF16, rank8_logit_std=4.0, index=4)
+    q, k, v = synth.make_qkv(w)
+    assert_close(run_gpu(q, k, v, w.scale, w.dtype, flags=tiles),
+                 oracle.attention(q, k, v, w.scale, w.dtype), f"tiles flag {tiles}")
 
 
 def test_increasing_logits_force_rescale_every_block(cuda_device):

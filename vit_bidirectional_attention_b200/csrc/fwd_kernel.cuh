@@ -110,6 +110,9 @@ constexpr unsigned kStatusTimeoutBase = 0x100;  // + site id
 // Test-only flag: the producer skips its first V load so that the consumer's
 // bounded wait runs out (exercises the timeout path without a fault).
 constexpr int kFlagSkipFirstVLoad = 1;
+// Test-only host flags: force two (or one) query tiles per CTA whatever the grid size.
+constexpr int kFlagForceTwoTiles = 2;
+constexpr int kFlagForceOneTile = 4;
 
 // ---------------------------------------------------------------- column chunks
 
@@ -156,8 +159,9 @@ struct alignas(64) FwdParams {
     CUtensorMap maps[3][3];  // [q, k, v][width class 64 / 32 / 16]
     void* out;
     int B, N, H, D;
-    int n_qpairs;   // ceil(N / 256): CTAs per (b, h)
-    int n_kblocks;  // ceil(N / 128)
+    int tiles_per_cta;  // query tiles a CTA owns: 2, or 1 when 2 would leave SMs idle
+    int n_qgroups;      // ceil(N / (128 * tiles_per_cta)): CTAs per (b, h)
+    int n_kblocks;      // ceil(N / 128)
     float scale_log2;
     int flags;
     unsigned long long timeout_ns;
@@ -440,14 +444,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // work item -> (b, h, query-tile pair); CTAs of one (b, h) are adjacent so
-    // they share K/V through L2.
-    const int qpair = blockIdx.x % p.n_qpairs;
-    const int bh = blockIdx.x / p.n_qpairs;
+    // work item -> (b, h, group of query tiles); CTAs of one (b, h) are
+    // adjacent so they share K/V through L2.
+    const int qgroup = blockIdx.x % p.n_qgroups;
+    const int bh = blockIdx.x / p.n_qgroups;
     const int h = bh % p.H;
     const int b = bh / p.H;
-    const int q0 = qpair * (kTilesPerCta * kTileRows);
-    const int ntiles = (q0 + kTileRows < p.N) ? 2 : 1;
+    const int q0 = qgroup * (p.tiles_per_cta * kTileRows);
+    const int ntiles = (p.tiles_per_cta == 2 && q0 + kTileRows < p.N) ? 2 : 1;
     const int nkb = p.n_kblocks;
     const uint64_t tmo = p.timeout_ns;
 

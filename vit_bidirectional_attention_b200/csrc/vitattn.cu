@@ -126,12 +126,13 @@ KernelFn pick_kernel(int dp, int dtype) {
 struct DeviceState {
     bool checked = false;
     bool is_sm100 = false;
+    int num_sms = 0;
     bool smem_set[9][2] = {};
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 
-int prepare_device(int dp, int dtype, KernelFn fn) {
+int prepare_device(int dp, int dtype, KernelFn fn, int* num_sms) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -145,9 +146,12 @@ int prepare_device(int dp, int dtype, KernelFn fn) {
         e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
         if (e != cudaSuccess) return cuda_fail(e);
         st.is_sm100 = (major == 10 && minor == 0);
+        e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
         st.checked = true;
     }
     if (!st.is_sm100) return VITATTN_ERR_DEVICE;
+    *num_sms = st.num_sms;
     bool& done = st.smem_set[dp / 16][dtype];
     if (!done) {
         e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
@@ -166,7 +170,8 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     const int dp = (int)((D + 15) / 16 * 16);
     KernelFn fn = pick_kernel(dp, dtype);
     if (!fn) return VITATTN_ERR_HEADDIM;
-    rc = prepare_device(dp, dtype, fn);
+    int num_sms = 0;
+    rc = prepare_device(dp, dtype, fn, &num_sms);
     if (rc) return rc;
 
     FwdParams prm;
@@ -185,13 +190,19 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     prm.N = (int)N;
     prm.H = (int)H;
     prm.D = (int)D;
-    prm.n_qpairs = (int)((N + 255) / 256);
+    // Two query tiles per CTA share each K/V block (fewer K/V reads, two
+    // softmax warpgroups in flight); one per CTA when two would leave SMs idle.
+    const uint64_t pairs = (uint64_t)B * (uint64_t)H * (uint64_t)((N + 255) / 256);
+    prm.tiles_per_cta = (N > 128 && pairs < (uint64_t)num_sms) ? 1 : 2;
+    if (flags & vitattn::kFlagForceTwoTiles) prm.tiles_per_cta = 2;
+    if (flags & vitattn::kFlagForceOneTile) prm.tiles_per_cta = 1;
+    prm.n_qgroups = (int)((N + 128 * prm.tiles_per_cta - 1) / (128 * prm.tiles_per_cta));
     prm.n_kblocks = (int)((N + 127) / 128);
     prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
     prm.flags = flags;
     prm.timeout_ns = kWaitTimeoutNs;
 
-    const unsigned grid = (unsigned)((uint64_t)B * (uint64_t)H * (uint64_t)prm.n_qpairs);
+    const unsigned grid = (unsigned)((uint64_t)B * (uint64_t)H * (uint64_t)prm.n_qgroups);
     void* args[1] = {&prm};
     cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid),
                                      dim3(vitattn::kThreads), args,
@@ -235,8 +246,9 @@ int vitattn_forward_checked(const void* q, const void* k, const void* v, void* o
 }
 
 // Test hook, deliberately absent from the public header: the checked entry
-// with kernel test flags (bit 0: the producer withholds the first V block so
-// that a bounded wait runs out and the timeout path is exercised).
+// with test flags (bit 0: the producer withholds the first V block so that a
+// bounded wait runs out and the timeout path is exercised; bit 1 / bit 2:
+// force two / one query tiles per CTA).
 VITATTN_API int vitattn_test_forward_flags(const void* q, const void* k, const void* v, void* out, int64_t B,
                                int64_t N, int64_t H, int64_t D, float scale, int dtype,
                                vitattn_stream_t stream, int flags) {
