@@ -42,6 +42,7 @@ def from_dev(t, dtype):
 
 FORCE_TWO_TILES = 2
 FORCE_ONE_TILE = 4
+TINY_GRID = 8
 
 
 def run_gpu(q, k, v, scale, dtype, flags=0):
@@ -155,6 +156,27 @@ def test_peaky_rescale_with_each_tile_mode(cuda_device, tiles):
     q, k, v = synth.make_qkv(w)
     assert_close(run_gpu(q, k, v, w.scale, w.dtype, flags=tiles),
                  oracle.attention(q, k, v, w.scale, w.dtype), f"tiles flag {tiles}")
+
+
+@pytest.mark.parametrize("tiles", [FORCE_TWO_TILES, FORCE_ONE_TILE])
+@pytest.mark.parametrize("D", [64, 80, 128])
+@pytest.mark.parametrize("N", [256, 768, 1000])
+def test_ctas_looping_over_many_items(cuda_device, N, D, tiles):
+    """At most three CTAs, each looping over many (b, h, query group) items:
+    the K/V ring, the S-buffer rotation, the per-tile block counters and the
+    Q buffers all carry over from item to item."""
+    q, k, v = synth.random_qkv(2, N, 3, D, synth.BF16, seed=5000 + N + D + tiles)
+    scale = 1.0 / math.sqrt(D)
+    assert_close(run_gpu(q, k, v, scale, synth.BF16, flags=tiles | TINY_GRID),
+                 oracle.attention(q, k, v, scale, synth.BF16), f"N={N} D={D} flags {tiles | TINY_GRID}")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_ctas_looping_over_items_with_rescales(cuda_device, D):
+    w = synth.Workload("peaky_items", 2, 1024, 3, D, synth.BF16, rank8_logit_std=4.0, index=4)
+    q, k, v = synth.make_qkv(w)
+    assert_close(run_gpu(q, k, v, w.scale, w.dtype, flags=FORCE_TWO_TILES | TINY_GRID),
+                 oracle.attention(q, k, v, w.scale, w.dtype))
 
 
 def test_increasing_logits_force_rescale_every_block(cuda_device):

@@ -89,8 +89,10 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max grows > 2^8
 
 // Barrier indices inside the barrier array.
-constexpr int kBarQFull = 0;                         // [2]
-constexpr int kBarKvFull = 2;                        // [kStages]
+constexpr int kMaxQBufs = 2;
+constexpr int kBarQFull = 0;                         // [kMaxQBufs][2 tiles] Q loaded
+constexpr int kBarQEmpty = kBarQFull + 2 * kMaxQBufs; // [kMaxQBufs][2 tiles] last S read it
+constexpr int kBarKvFull = kBarQEmpty + 2 * kMaxQBufs;  // [kStages]
 constexpr int kBarKvEmpty = kBarKvFull + kStages;    // [kStages]
 constexpr int kMaxSBufs = 3;
 constexpr int kBarSFull = kBarKvEmpty + kStages;     // [kMaxSBufs] one per S buffer
@@ -100,8 +102,9 @@ constexpr int kBarSFull = kBarKvEmpty + kStages;     // [kMaxSBufs] one per S bu
 // ahead of its waiter; block j+2 needs P.V of block j first, so two cannot.
 constexpr int kBarPFull = kBarSFull + kMaxSBufs;
 constexpr int kBarOReady = kBarPFull + 4;            // [2] per tile: a P.V product finished
-constexpr int kBarOFull = kBarOReady + 2;            // [2] per tile: the last P.V finished
-constexpr int kBarDrain = kBarOFull + 2;             // [1]
+constexpr int kBarOFull = kBarOReady + 2;            // [2] per tile: the item's last P.V finished
+constexpr int kBarOEmpty = kBarOFull + 2;            // [2] per tile: the epilogue has read O
+constexpr int kBarDrain = kBarOEmpty + 2;            // [1]
 constexpr int kNumBars = kBarDrain + 1;
 
 // Status codes written to g_vitattn_status (0 = fine).
@@ -110,9 +113,11 @@ constexpr unsigned kStatusTimeoutBase = 0x100;  // + site id
 // Test-only flag: the producer skips its first V load so that the consumer's
 // bounded wait runs out (exercises the timeout path without a fault).
 constexpr int kFlagSkipFirstVLoad = 1;
-// Test-only host flags: force two (or one) query tiles per CTA whatever the grid size.
+// Test-only host flags: force two (or one) query tiles per CTA whatever the grid
+// size; run the whole problem on at most three CTAs (many work items each).
 constexpr int kFlagForceTwoTiles = 2;
 constexpr int kFlagForceOneTile = 4;
+constexpr int kFlagTinyGrid = 8;
 
 // ---------------------------------------------------------------- column chunks
 
@@ -151,16 +156,20 @@ __host__ __device__ constexpr int active_s_buffers(int ns, int ntiles) {
 // S(t, j) already proves P.V(t, j-1) done and the separate "P.V done"
 // barrier (one extra tcgen05.commit per product) is not needed.
 __host__ __device__ constexpr bool pv_done_needed(int ns, int ntiles) { return ns != ntiles; }
+// Q tiles are double-buffered (the next work item's Q loads while the current
+// one runs) when that fits in shared memory, i.e. up to DP = 112.
+__host__ __device__ constexpr int q_buffers(int dp) { return dp <= 112 ? 2 : 1; }
 __host__ __device__ constexpr int smem_bytes(int dp) {
-    return (kTilesPerCta + kStages) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
+    return (q_buffers(dp) * kTilesPerCta + kStages) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
 }
 
 struct alignas(64) FwdParams {
     CUtensorMap maps[3][3];  // [q, k, v][width class 64 / 32 / 16]
     void* out;
     int B, N, H, D;
-    int tiles_per_cta;  // query tiles a CTA owns: 2, or 1 when 2 would leave SMs idle
-    int n_qgroups;      // ceil(N / (128 * tiles_per_cta)): CTAs per (b, h)
+    int tiles_per_cta;  // query tiles a work item owns: 2, or 1 when 2 would leave SMs idle
+    int n_qgroups;      // ceil(N / (128 * tiles_per_cta)): work items per (b, h)
+    int n_items;        // B * H * n_qgroups; a CTA takes items blockIdx.x + k * gridDim.x
     int n_kblocks;      // ceil(N / 128)
     float scale_log2;
     int flags;
@@ -429,34 +438,50 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     constexpr int NCH = chunk_count(DP);
     static_assert(DP % 16 == 0 && DP >= 16 && DP <= 128, "head dim padding");
 
+    constexpr int NQ = q_buffers(DP);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* const base_ptr = smem_raw + (base - raw);
-    const uint32_t sQ = base;
-    const uint32_t sKV = base + kTilesPerCta * TILE;
-    const uint32_t sBar = base + (kTilesPerCta + kStages) * TILE;
+    const uint32_t sQ = base;  // [NQ][2 tiles]
+    const uint32_t sKV = base + NQ * kTilesPerCta * TILE;
+    const uint32_t sBar = base + (NQ * kTilesPerCta + kStages) * TILE;
     uint32_t* const tmem_holder =
-        reinterpret_cast<uint32_t*>(base_ptr + (kTilesPerCta + kStages) * TILE + kNumBars * 8);
+        reinterpret_cast<uint32_t*>(base_ptr + (NQ * kTilesPerCta + kStages) * TILE + kNumBars * 8);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
     auto bar = [&](int i) -> uint32_t { return sBar + 8u * (uint32_t)i; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // work item -> (b, h, group of query tiles); CTAs of one (b, h) are
-    // adjacent so they share K/V through L2.
-    const int qgroup = blockIdx.x % p.n_qgroups;
-    const int bh = blockIdx.x / p.n_qgroups;
-    const int h = bh % p.H;
-    const int b = bh / p.H;
-    const int q0 = qgroup * (p.tiles_per_cta * kTileRows);
-    const int ntiles = (p.tiles_per_cta == 2 && q0 + kTileRows < p.N) ? 2 : 1;
+    // Work items: (b, h, group of query tiles), numbered so that the items of
+    // one (b, h) are adjacent and the CTAs running at once share K/V in L2.
+    // This CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...; the host
+    // launches fewer CTAs than items only when every item has the same number
+    // of query tiles, so T below holds for all of this CTA's items.
+    struct Item {
+        int b, h, q0, nt;
+    };
+    auto item_of = [&](int i) -> Item {
+        Item it;
+        const int qg = i % p.n_qgroups;
+        const int bh = i / p.n_qgroups;
+        it.h = bh % p.H;
+        it.b = bh / p.H;
+        it.q0 = qg * (p.tiles_per_cta * kTileRows);
+        it.nt = (p.tiles_per_cta == 2 && it.q0 + kTileRows < p.N) ? 2 : 1;
+        return it;
+    };
+    const int n_my = (p.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int T = item_of(blockIdx.x).nt;
     const int nkb = p.n_kblocks;
     const uint64_t tmo = p.timeout_ns;
 
     if (threadIdx.x == 0) {
-        for (int t = 0; t < 2; ++t) ptx::mbar_init(bar(kBarQFull + t), 1);
+        for (int i = 0; i < 2 * kMaxQBufs; ++i) {
+            ptx::mbar_init(bar(kBarQFull + i), 1);
+            ptx::mbar_init(bar(kBarQEmpty + i), 1);
+        }
         for (int s = 0; s < kStages; ++s) {
             ptx::mbar_init(bar(kBarKvFull + s), 1);
             ptx::mbar_init(bar(kBarKvEmpty + s), 1);
@@ -467,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             ptx::mbar_init(bar(kBarPFull + 2 * t + 1), 4 * 32);
             ptx::mbar_init(bar(kBarOReady + t), 1);
             ptx::mbar_init(bar(kBarOFull + t), 1);
+            ptx::mbar_init(bar(kBarOEmpty + t), 4 * 32);
         }
         ptx::mbar_init(bar(kBarDrain), 1);
         *abort_flag = 0;
@@ -493,47 +519,57 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
                 for (int m = 0; m < 3; ++m)
                     ptx::prefetch_tensormap(&p.maps[m][width_class(chunk_width(DP, c))]);
-            for (int t = 0; t < ntiles; ++t) {
-                ptx::mbar_arrive_expect_tx(bar(kBarQFull + t), TILE);
-#pragma unroll
-                for (int c = 0; c < NCH; ++c)
-                    ptx::tma_load_4d(sQ + t * TILE + 256 * chunk_col(DP, c),
-                                     &p.maps[0][width_class(chunk_width(DP, c))], chunk_col(DP, c),
-                                     h, q0 + t * kTileRows, b, bar(kBarQFull + t));
-            }
-            int issued = 0;
+            int r = 0;         // K/V ring entries issued so far (K_j, V_j of each item in turn)
+            int q_last[2] = {-1, -1};  // last item whose Q tile t was issued
             bool ok = true;
-            for (int j = 0; j < nkb && ok; ++j) {
-                for (int kv = 0; kv < 2; ++kv) {
-                    const int idx = 2 * j + kv;
-                    const int slot = idx % kStages;
-                    const uint32_t phase = (uint32_t)(idx / kStages) & 1u;
-                    if (!wait_one(bar(kBarKvEmpty + slot), phase ^ 1u, abort_flag, tmo, 1)) {
+            for (int k = 0; k < n_my && ok; ++k) {
+                const Item it = item_of((int)blockIdx.x + k * (int)gridDim.x);
+                const int qb = k % NQ;
+                for (int t = 0; t < T && ok; ++t) {
+                    // Q buffer qb of tile t was last read by the S products of item k - NQ
+                    if (k >= NQ && !wait_one(bar(kBarQEmpty + 2 * qb + t), (uint32_t)((k / NQ) - 1) & 1u,
+                                             abort_flag, tmo, 12)) {
                         ok = false;
                         break;
                     }
-                    if (kv == 1 && j == 0 && (p.flags & kFlagSkipFirstVLoad)) {
-                        issued = idx + 1;
-                        continue;  // test-only: never fill this slot
-                    }
-                    ptx::mbar_arrive_expect_tx(bar(kBarKvFull + slot), TILE);
+                    ptx::mbar_arrive_expect_tx(bar(kBarQFull + 2 * qb + t), TILE);
 #pragma unroll
                     for (int c = 0; c < NCH; ++c)
-                        ptx::tma_load_4d(sKV + slot * TILE + 256 * chunk_col(DP, c),
-                                         &p.maps[1 + kv][width_class(chunk_width(DP, c))],
-                                         chunk_col(DP, c), h, j * kBlockKeys, b,
-                                         bar(kBarKvFull + slot));
-                    issued = idx + 1;
+                        ptx::tma_load_4d(sQ + (qb * kTilesPerCta + t) * TILE + 256 * chunk_col(DP, c),
+                                         &p.maps[0][width_class(chunk_width(DP, c))], chunk_col(DP, c),
+                                         it.h, it.q0 + t * kTileRows, it.b, bar(kBarQFull + 2 * qb + t));
+                    q_last[t] = k;
+                }
+
+                for (int j = 0; j < nkb && ok; ++j) {
+                    for (int kv = 0; kv < 2; ++kv, ++r) {
+                        const int slot = r % kStages;
+                        const uint32_t phase = (uint32_t)(r / kStages) & 1u;
+                        if (!wait_one(bar(kBarKvEmpty + slot), phase ^ 1u, abort_flag, tmo, 1)) {
+                            ok = false;
+                            break;
+                        }
+                        if (r == 1 && (p.flags & kFlagSkipFirstVLoad)) continue;  // test-only
+                        ptx::mbar_arrive_expect_tx(bar(kBarKvFull + slot), TILE);
+#pragma unroll
+                        for (int c = 0; c < NCH; ++c)
+                            ptx::tma_load_4d(sKV + slot * TILE + 256 * chunk_col(DP, c),
+                                             &p.maps[1 + kv][width_class(chunk_width(DP, c))],
+                                             chunk_col(DP, c), it.h, j * kBlockKeys, it.b,
+                                             bar(kBarKvFull + slot));
+                    }
                 }
             }
             {
                 // let every copy this CTA started land before the CTA exits (in a
                 // normal run they all have; after an abort some may not have been
-                // waited for).  The last fill of each slot is its latest phase, so
-                // its parity is unambiguous whether or not it was consumed.
+                // waited for).  The last fill of each buffer or slot is its latest
+                // phase, so its parity is unambiguous whether or not it was consumed.
                 const uint64_t drain_ns = 200000000ull;
-                for (int t = 0; t < ntiles; ++t) wait_drain(bar(kBarQFull + t), 0, drain_ns);
-                for (int idx = issued - 1; idx >= 0 && idx >= issued - kStages; --idx) {
+                for (int t = 0; t < T; ++t)
+                    for (int k = q_last[t]; k >= 0 && k > q_last[t] - NQ; --k)
+                        wait_drain(bar(kBarQFull + 2 * (k % NQ) + t), (uint32_t)(k / NQ) & 1u, drain_ns);
+                for (int idx = r - 1; idx >= 0 && idx >= r - kStages; --idx) {
                     if ((p.flags & kFlagSkipFirstVLoad) && idx == 1) continue;
                     wait_drain(bar(kBarKvFull + idx % kStages), (uint32_t)(idx / kStages) & 1u,
                                drain_ns);
@@ -550,12 +586,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             constexpr uint32_t idS = idesc_f16(kBF16, kBlockKeys, false);
             constexpr int NS = s_buffers(DP);
             constexpr int OC = o_cols(DP);
-            auto mma_s = [&](int t, int slot, int buf) {
+            auto mma_s = [&](int qtile, int slot, int buf) {
                 const uint32_t d = tmem + (uint32_t)(buf * kBlockKeys);
 #pragma unroll
                 for (int c = 0; c < NCH; ++c) {
                     const int w = chunk_width(DP, c);
-                    const uint64_t qd = sdesc(sQ + t * TILE + 256 * chunk_col(DP, c), 16,
+                    const uint64_t qd = sdesc(sQ + qtile * TILE + 256 * chunk_col(DP, c), 16,
                                               16u * (uint32_t)w, swizzle_code(w));
                     const uint64_t kd = sdesc(sKV + slot * TILE + 256 * chunk_col(DP, c), 16,
                                               16u * (uint32_t)w, swizzle_code(w));
@@ -601,54 +637,69 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             // K_j and V_j occupy ring entries 2j and 2j+1 (the producer's order).
             auto kv_slot = [](int idx) { return idx % kStages; };
             auto kv_parity = [](int idx) { return (uint32_t)(idx / kStages) & 1u; };
-            const int T = ntiles;
-            const int total = T * nkb;
+            const int total = n_my * T * nkb;  // units of all this CTA's items
             const int ns = active_s_buffers(NS, T);
             const bool track_pv = pv_done_needed(ns, T);
             // A cursor walks the units s = T*j + t in order, keeping (t, j) and the
             // S buffer s mod ns without divisions (this thread is on the critical path).
             struct Cursor {
-                int t, j, buf;
+                int t, j, k, g, buf;  // tile, block, item (local index), block count g = k*nkb + j
             };
             auto advance = [&](Cursor& c) {
                 if (++c.t == T) {
                     c.t = 0;
-                    ++c.j;
+                    ++c.g;
+                    if (++c.j == nkb) {
+                        c.j = 0;
+                        ++c.k;
+                    }
                 }
                 if (++c.buf == ns) c.buf = 0;
             };
             // S for one unit into its buffer; K_j is waited for by its first unit
             // and released after its last.
             auto issue_s = [&](const Cursor& c) -> bool {
-                if (c.t == 0) {
-                    if (!wait_one(bar(kBarKvFull + kv_slot(2 * c.j)), kv_parity(2 * c.j), abort_flag, tmo, 3))
+                const int qb = c.k % NQ;
+                if (c.j == 0) {  // first S of this tile in this item: its Q tile
+                    if (!wait_one(bar(kBarQFull + 2 * qb + c.t), (uint32_t)(c.k / NQ) & 1u, abort_flag, tmo, 2))
                         return false;
                     ptx::tc_fence_after();
                 }
-                mma_s(c.t, kv_slot(2 * c.j), c.buf);
+                if (c.t == 0) {
+                    if (!wait_one(bar(kBarKvFull + kv_slot(2 * c.g)), kv_parity(2 * c.g), abort_flag, tmo, 3))
+                        return false;
+                    ptx::tc_fence_after();
+                }
+                mma_s(qb * kTilesPerCta + c.t, kv_slot(2 * c.g), c.buf);
                 ptx::mma_commit(bar(kBarSFull + c.buf));
-                if (c.t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * c.j)));
+                if (c.t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * c.g)));
+                if (c.j == nkb - 1) ptx::mma_commit(bar(kBarQEmpty + 2 * qb + c.t));
                 return true;
             };
             // O_t += P V_j; V_j is waited for by its first unit and released after its last.
             auto issue_pv = [&](const Cursor& c) -> bool {
-                const int t = c.t, j = c.j;
+                const int t = c.t, j = c.j, g = c.g;
                 if (t == 0 &&
-                    !wait_one(bar(kBarKvFull + kv_slot(2 * j + 1)), kv_parity(2 * j + 1), abort_flag, tmo, 4))
+                    !wait_one(bar(kBarKvFull + kv_slot(2 * g + 1)), kv_parity(2 * g + 1), abort_flag, tmo, 4))
                     return false;
-                if (!wait_one(bar(kBarPFull + 2 * t + (j & 1)), (uint32_t)(j >> 1) & 1u, abort_flag, tmo, 5))
+                // the first product of an item overwrites O_t: the previous item's
+                // epilogue must have read it out
+                if (j == 0 && c.k > 0 &&
+                    !wait_one(bar(kBarOEmpty + t), (uint32_t)(c.k - 1) & 1u, abort_flag, tmo, 13))
+                    return false;
+                if (!wait_one(bar(kBarPFull + 2 * t + (g & 1)), (uint32_t)(g >> 1) & 1u, abort_flag, tmo, 5))
                     return false;
                 ptx::tc_fence_after();
-                mma_pv(t, kv_slot(2 * j + 1), c.buf, j > 0);
+                mma_pv(t, kv_slot(2 * g + 1), c.buf, j > 0);
                 if (track_pv) ptx::mma_commit(bar(kBarOReady + t));
-                if (t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * j + 1)));
+                if (t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * g + 1)));
+                if (j == nkb - 1) ptx::mma_commit(bar(kBarOFull + t));
                 return true;
             };
 
             bool ok = true;
-            for (int t = 0; t < T && ok; ++t) ok = wait_one(bar(kBarQFull + t), 0, abort_flag, tmo, 2);
-            Cursor cs{0, 0, 0};  // next unit whose S is issued
-            Cursor cp{0, 0, 0};  // next unit whose P.V is issued
+            Cursor cs{0, 0, 0, 0, 0};  // next unit whose S is issued
+            Cursor cp{0, 0, 0, 0, 0};  // next unit whose P.V is issued
             int issued_s = 0;
             for (; issued_s < ns && issued_s < total && ok; ++issued_s) {
                 ok = issue_s(cs);
@@ -663,9 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     ++issued_s;
                 }
             }
-            if (ok) {
-                for (int t = 0; t < ntiles; ++t) ptx::mma_commit(bar(kBarOFull + t));
-            } else {
+            if (!ok) {
                 // every MMA issued so far must finish before TMEM is freed
                 ptx::mma_commit(bar(kBarDrain));
                 wait_drain(bar(kBarDrain), 0, 200000000ull);
@@ -678,25 +727,29 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         // ------------------------------------------------------------ softmax
         const int t = warp >> 2;
         const int wq = warp & 3;
-        if (t < ntiles) {
+        if (t < T) {
             constexpr int NS = s_buffers(DP);
-            const int ns = active_s_buffers(NS, ntiles);
+            const int ns = active_s_buffers(NS, T);
             const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
             const uint32_t tO = tmem + lane_base + (uint32_t)(NS * kBlockKeys + t * o_cols(DP));
-            const int row = q0 + t * kTileRows + wq * 32 + lane;
             const float c2 = p.scale_log2;
             const bool neg = c2 < 0.f;
+            bool ok = true;
+            // unit = T*g + t (g = blocks of this tile so far, over all items) lives
+            // in S buffer unit % ns, as phase unit / ns of that buffer's barrier;
+            // both advance by T units per block.
+            int sbuf = t % ns, sphase = t / ns;
+            int g = 0;
+            for (int k = 0; k < n_my && ok; ++k) {
+            const Item it = item_of((int)blockIdx.x + k * (int)gridDim.x);
+            const int row = it.q0 + t * kTileRows + wq * 32 + lane;
             float m_used = -INFINITY;
             float l = 0.f;
-            bool ok = true;
-            // unit = ntiles*j + t lives in S buffer unit % ns, as phase unit / ns of
-            // that buffer's barrier; both advance by ntiles units per block.
-            int sbuf = t % ns, sphase = t / ns;
-            for (int j = 0; j < nkb; ++j) {
+            for (int j = 0; j < nkb; ++j, ++g) {
                 const uint32_t tS = tmem + lane_base + (uint32_t)(sbuf * kBlockKeys);
                 const uint32_t s_bar = bar(kBarSFull + sbuf);
                 const uint32_t s_par = (uint32_t)sphase & 1u;
-                sbuf += ntiles;
+                sbuf += T;
                 if (sbuf >= ns) {
                     sbuf -= ns;
                     ++sphase;
@@ -739,8 +792,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 // wait for it (phase j-1 of the per-tile "P.V done" barrier; the phase
                 // of block j-2 has completed by now, so the parity is unambiguous).
                 if (j > 0 && __any_sync(0xffffffffu, need)) {
-                    if (pv_done_needed(ns, ntiles) &&
-                        !wait_warp(bar(kBarOReady + t), (uint32_t)(j - 1) & 1u, abort_flag, tmo, 11)) {
+                    if (pv_done_needed(ns, T) &&
+                        !wait_warp(bar(kBarOReady + t), (uint32_t)(g - 1) & 1u, abort_flag, tmo, 11)) {
                         ok = false;
                         break;
                     }
@@ -749,14 +802,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(bar(kBarPFull + 2 * t + (j & 1)));
+                ptx::mbar_arrive(bar(kBarPFull + 2 * t + (g & 1)));
             }
-            if (ok) ok = wait_warp(bar(kBarOFull + t), 0, abort_flag, tmo, 8);
+            if (ok) ok = wait_warp(bar(kBarOFull + t), (uint32_t)k & 1u, abort_flag, tmo, 8);
             if (ok) {
                 ptx::tc_fence_after();
                 uint8_t* orow = reinterpret_cast<uint8_t*>(p.out) +
-                                ((((size_t)b * p.N + (size_t)min(row, p.N - 1)) * p.H + h) * p.D) * 2;
+                                ((((size_t)it.b * p.N + (size_t)min(row, p.N - 1)) * p.H + it.h) * p.D) * 2;
                 store_row<DP, kBF16>(tO, 1.f / l, orow, row < p.N, p.D);
+                // O_t has been read (store_row waits for each load): the next
+                // item's first P.V may overwrite it
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(bar(kBarOEmpty + t));
+            }
             }
         }
     }

@@ -197,12 +197,21 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     if (flags & vitattn::kFlagForceTwoTiles) prm.tiles_per_cta = 2;
     if (flags & vitattn::kFlagForceOneTile) prm.tiles_per_cta = 1;
     prm.n_qgroups = (int)((N + 128 * prm.tiles_per_cta - 1) / (128 * prm.tiles_per_cta));
+    prm.n_items = (int)((uint64_t)B * (uint64_t)H * (uint64_t)prm.n_qgroups);
     prm.n_kblocks = (int)((N + 127) / 128);
     prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
     prm.flags = flags;
     prm.timeout_ns = kWaitTimeoutNs;
 
-    const unsigned grid = (unsigned)((uint64_t)B * (uint64_t)H * (uint64_t)prm.n_qgroups);
+    // Persistent grid (one CTA per SM, each looping over work items) when there
+    // are more items than SMs, the items are short enough (at most 32 key
+    // blocks) for the per-CTA start-up and epilogue to matter, and every item
+    // has the same number of query tiles (all have two unless the last group
+    // of a head is a single tile); otherwise one CTA per item.
+    const bool uniform = prm.tiles_per_cta == 1 || (N % 256 == 0 || N % 256 > 128);
+    unsigned grid = (unsigned)prm.n_items;
+    if (uniform && prm.n_items > num_sms && prm.n_kblocks <= 32) grid = (unsigned)num_sms;
+    if (uniform && (flags & vitattn::kFlagTinyGrid) && grid > 3u) grid = 3u;
     void* args[1] = {&prm};
     cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid),
                                      dim3(vitattn::kThreads), args,
@@ -248,7 +257,8 @@ int vitattn_forward_checked(const void* q, const void* k, const void* v, void* o
 // Test hook, deliberately absent from the public header: the checked entry
 // with test flags (bit 0: the producer withholds the first V block so that a
 // bounded wait runs out and the timeout path is exercised; bit 1 / bit 2:
-// force two / one query tiles per CTA).
+// force two / one query tiles per work item; bit 3: at most three CTAs, each
+// looping over many work items).
 VITATTN_API int vitattn_test_forward_flags(const void* q, const void* k, const void* v, void* out, int64_t B,
                                int64_t N, int64_t H, int64_t D, float scale, int dtype,
                                vitattn_stream_t stream, int flags) {
