@@ -157,10 +157,11 @@ __host__ __device__ constexpr int active_s_buffers(int ns, int ntiles) {
 // barrier (one extra tcgen05.commit per product) is not needed.
 __host__ __device__ constexpr bool pv_done_needed(int ns, int ntiles) { return ns != ntiles; }
 // Q tiles are double-buffered (the next work item's Q loads while the current
-// one runs) when that fits in shared memory, i.e. up to DP = 112.
-__host__ __device__ constexpr int q_buffers(int dp) { return dp <= 112 ? 2 : 1; }
-__host__ __device__ constexpr int smem_bytes(int dp) {
-    return (q_buffers(dp) * kTilesPerCta + kStages) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
+// one runs) when a CTA loops over items and that fits in shared memory, i.e.
+// up to DP = 112.
+__host__ __device__ constexpr int q_buffers(int dp, bool loop) { return (loop && dp <= 112) ? 2 : 1; }
+__host__ __device__ constexpr int smem_bytes(int dp, bool loop) {
+    return (q_buffers(dp, loop) * kTilesPerCta + kStages) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
 }
 
 struct alignas(64) FwdParams {
@@ -432,13 +433,15 @@ __device__ __forceinline__ void store_row(uint32_t tO, float inv_l, uint8_t* oro
 
 // ---------------------------------------------------------------- the kernel
 
-template <int DP, bool kBF16>
+// kLoop: the CTA loops over work items (grid smaller than the item count);
+// without it every CTA owns exactly one item and the item loops fold away.
+template <int DP, bool kBF16, bool kLoop>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
     constexpr int TILE = tile_bytes(DP);
     constexpr int NCH = chunk_count(DP);
     static_assert(DP % 16 == 0 && DP >= 16 && DP <= 128, "head dim padding");
 
-    constexpr int NQ = q_buffers(DP);
+    constexpr int NQ = q_buffers(DP, kLoop);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -472,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         it.nt = (p.tiles_per_cta == 2 && it.q0 + kTileRows < p.N) ? 2 : 1;
         return it;
     };
-    const int n_my = (p.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int n_my = kLoop ? (p.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 1;
     const int T = item_of(blockIdx.x).nt;
     const int nkb = p.n_kblocks;
     const uint64_t tmo = p.timeout_ns;
@@ -527,8 +530,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 const int qb = k % NQ;
                 for (int t = 0; t < T && ok; ++t) {
                     // Q buffer qb of tile t was last read by the S products of item k - NQ
-                    if (k >= NQ && !wait_one(bar(kBarQEmpty + 2 * qb + t), (uint32_t)((k / NQ) - 1) & 1u,
-                                             abort_flag, tmo, 12)) {
+                    if (kLoop && k >= NQ &&
+                        !wait_one(bar(kBarQEmpty + 2 * qb + t), (uint32_t)((k / NQ) - 1) & 1u, abort_flag,
+                                  tmo, 12)) {
                         ok = false;
                         break;
                     }
@@ -673,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 mma_s(qb * kTilesPerCta + c.t, kv_slot(2 * c.g), c.buf);
                 ptx::mma_commit(bar(kBarSFull + c.buf));
                 if (c.t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * c.g)));
-                if (c.j == nkb - 1) ptx::mma_commit(bar(kBarQEmpty + 2 * qb + c.t));
+                if (kLoop && c.j == nkb - 1) ptx::mma_commit(bar(kBarQEmpty + 2 * qb + c.t));
                 return true;
             };
             // O_t += P V_j; V_j is waited for by its first unit and released after its last.
@@ -684,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     return false;
                 // the first product of an item overwrites O_t: the previous item's
                 // epilogue must have read it out
-                if (j == 0 && c.k > 0 &&
+                if (kLoop && j == 0 && c.k > 0 &&
                     !wait_one(bar(kBarOEmpty + t), (uint32_t)(c.k - 1) & 1u, abort_flag, tmo, 13))
                     return false;
                 if (!wait_one(bar(kBarPFull + 2 * t + (g & 1)), (uint32_t)(g >> 1) & 1u, abort_flag, tmo, 5))
@@ -812,8 +816,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 store_row<DP, kBF16>(tO, 1.f / l, orow, row < p.N, p.D);
                 // O_t has been read (store_row waits for each load): the next
                 // item's first P.V may overwrite it
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(bar(kBarOEmpty + t));
+                if (kLoop) {
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(bar(kBarOEmpty + t));
+                }
             }
             }
         }

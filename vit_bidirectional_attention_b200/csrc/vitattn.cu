@@ -101,22 +101,23 @@ bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t N
 
 using KernelFn = void (*)(FwdParams);
 
-template <int DP, bool BF>
-KernelFn kernel_of() {
-    return vitattn::fwd_kernel<DP, BF>;
+template <int DP>
+KernelFn kernel_of(bool bf, bool loop) {
+    if (bf) return loop ? vitattn::fwd_kernel<DP, true, true> : vitattn::fwd_kernel<DP, true, false>;
+    return loop ? vitattn::fwd_kernel<DP, false, true> : vitattn::fwd_kernel<DP, false, false>;
 }
 
-KernelFn pick_kernel(int dp, int dtype) {
+KernelFn pick_kernel(int dp, int dtype, bool loop) {
     const bool bf = dtype == VITATTN_BF16;
     switch (dp) {
-        case 16: return bf ? kernel_of<16, true>() : kernel_of<16, false>();
-        case 32: return bf ? kernel_of<32, true>() : kernel_of<32, false>();
-        case 48: return bf ? kernel_of<48, true>() : kernel_of<48, false>();
-        case 64: return bf ? kernel_of<64, true>() : kernel_of<64, false>();
-        case 80: return bf ? kernel_of<80, true>() : kernel_of<80, false>();
-        case 96: return bf ? kernel_of<96, true>() : kernel_of<96, false>();
-        case 112: return bf ? kernel_of<112, true>() : kernel_of<112, false>();
-        case 128: return bf ? kernel_of<128, true>() : kernel_of<128, false>();
+        case 16: return kernel_of<16>(bf, loop);
+        case 32: return kernel_of<32>(bf, loop);
+        case 48: return kernel_of<48>(bf, loop);
+        case 64: return kernel_of<64>(bf, loop);
+        case 80: return kernel_of<80>(bf, loop);
+        case 96: return kernel_of<96>(bf, loop);
+        case 112: return kernel_of<112>(bf, loop);
+        case 128: return kernel_of<128>(bf, loop);
         default: return nullptr;
     }
 }
@@ -127,12 +128,13 @@ struct DeviceState {
     bool checked = false;
     bool is_sm100 = false;
     int num_sms = 0;
-    bool smem_set[9][2] = {};
+    bool smem_set[9][2][2] = {};
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 
-int prepare_device(int dp, int dtype, KernelFn fn, int* num_sms) {
+// Architecture check and SM count, once per device.
+int device_info(int* num_sms) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -152,11 +154,20 @@ int prepare_device(int dp, int dtype, KernelFn fn, int* num_sms) {
     }
     if (!st.is_sm100) return VITATTN_ERR_DEVICE;
     *num_sms = st.num_sms;
-    bool& done = st.smem_set[dp / 16][dtype];
+    return VITATTN_OK;
+}
+
+// The dynamic shared-memory limit of one kernel instantiation, raised once per device.
+int ensure_smem(int dp, int dtype, bool loop, KernelFn fn) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    std::lock_guard<std::mutex> lock(g_mu);
+    bool& done = g_dev[dev].smem_set[dp / 16][dtype][loop ? 1 : 0];
     if (!done) {
         e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 vitattn::smem_bytes(dp));
+                                 vitattn::smem_bytes(dp, loop));
         if (e != cudaSuccess) return cuda_fail(e);
         done = true;
     }
@@ -168,10 +179,8 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     int rc = check_args(q, k, v, out, B, N, H, D, scale, dtype);
     if (rc) return rc;
     const int dp = (int)((D + 15) / 16 * 16);
-    KernelFn fn = pick_kernel(dp, dtype);
-    if (!fn) return VITATTN_ERR_HEADDIM;
     int num_sms = 0;
-    rc = prepare_device(dp, dtype, fn, &num_sms);
+    rc = device_info(&num_sms);
     if (rc) return rc;
 
     FwdParams prm;
@@ -212,10 +221,16 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     unsigned grid = (unsigned)prm.n_items;
     if (uniform && prm.n_items > num_sms && prm.n_kblocks <= 32) grid = (unsigned)num_sms;
     if (uniform && (flags & vitattn::kFlagTinyGrid) && grid > 3u) grid = 3u;
+    const bool loop = grid < (unsigned)prm.n_items;
+
+    KernelFn fn = pick_kernel(dp, dtype, loop);
+    if (!fn) return VITATTN_ERR_HEADDIM;
+    rc = ensure_smem(dp, dtype, loop, fn);
+    if (rc) return rc;
     void* args[1] = {&prm};
     cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid),
                                      dim3(vitattn::kThreads), args,
-                                     (size_t)vitattn::smem_bytes(dp), stream);
+                                     (size_t)vitattn::smem_bytes(dp, loop), stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return VITATTN_OK;
 }
