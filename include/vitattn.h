@@ -22,8 +22,13 @@
  * contiguous: element (b, i, h, d) at ((b*N + i)*H + h)*D + d.  That is the
  * layout a QKV linear produces once its output is split into three.
  * Lq = Lk = N (self-attention).  out has the dtype of the inputs; products
- * and sums accumulate in fp32, probabilities are rounded to the input dtype
- * before the P.V product.
+ * and sums accumulate in fp32.  The probabilities enter the P.V product as
+ * f16 for both dtypes (f16 carries three more mantissa bits than bf16), and
+ * for bf16 inputs V is converted to f16 for that product: exact for
+ * |v| < 65536 outside f16's subnormal range (|v| < 2^-14, where the absolute
+ * error stays below 2^-25).  A bf16 V value of magnitude >= 65536 (or an
+ * infinite one) becomes inf in that product; vitattn_forward_checked reports
+ * it as VITATTN_ERR_RANGE.
  *
  * Ownership.  The caller owns every buffer.  The library allocates no device
  * memory, keeps no reference to any buffer after a call returns, and never
@@ -78,7 +83,8 @@ enum vitattn_status {
     VITATTN_ERR_CUDA = -7,    /* the CUDA runtime or driver returned an error */
     VITATTN_ERR_TIMEOUT = -8, /* a bounded in-kernel wait ran out (checked entry only) */
     VITATTN_ERR_SCALE = -9,   /* scale is NaN or infinite */
-    VITATTN_ERR_DEVICE = -10  /* the current device is not an sm_100 GPU */
+    VITATTN_ERR_DEVICE = -10, /* the current device is not an sm_100 GPU */
+    VITATTN_ERR_RANGE = -11   /* a bf16 V value has |v| >= 65536 (checked entry only) */
 };
 
 /*
@@ -98,9 +104,12 @@ VITATTN_API int vitattn_forward(const void* q, const void* k, const void* v, voi
 
 /*
  * vitattn_forward_checked -- vitattn_forward, then a stream synchronisation
- * and a read of the kernel's status word.  Returns VITATTN_ERR_TIMEOUT when a
- * bounded in-kernel wait ran out, VITATTN_ERR_CUDA when the stream reported
- * an error.  Meant for tests and debugging: it blocks the calling thread.
+ * and a read of the kernel's status words.  Returns VITATTN_ERR_TIMEOUT when a
+ * bounded in-kernel wait ran out, VITATTN_ERR_RANGE when a bf16 V value was
+ * outside the f16 range of the P.V product (out then holds inf or NaN in the
+ * affected rows), VITATTN_ERR_CUDA when the stream reported an error.  Meant
+ * for tests and debugging: it blocks the calling thread.  Checked calls that
+ * overlap in time (several streams or threads) share the status words.
  */
 VITATTN_API int vitattn_forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B,
                             int64_t N, int64_t H, int64_t D, float scale, int dtype,

@@ -275,3 +275,67 @@ def test_errors_on_device_do_not_launch(cuda_device):
     assert e.value.status == -6
     assert vitattn.forward_ptr(t.data_ptr() + 2, t.data_ptr(), t.data_ptr(), t.data_ptr() + 4096,
                                1, 1, 1, 64, 1.0, 0) == -5
+
+
+# ------------------------------------------------------------------ f16 P.V product
+
+def _v_in_f16_normal_range(shape, seed):
+    """bf16 V with every nonzero |v| in [2^-10, 3.984375]: exact in f16, and
+    still exact in f16 after scaling by 2^14 (largest |v| 65280 < 2^16)."""
+    v = np.random.Generator(np.random.PCG64(seed)).standard_normal(shape).astype(np.float32)
+    v = np.clip(v, -3.984375, 3.984375)
+    v[np.abs(v) < 2.0 ** -10] = 0.0
+    return synth.round_to_bits(v, synth.BF16)
+
+
+@pytest.mark.parametrize("D", [64, 80, 128])
+def test_v_scaled_to_top_of_f16_range_scales_output_exactly(cuda_device, D):
+    """Scaling V by 2^14 scales every product and sum of the P.V step by a
+    power of two (no rounding changes) up to |v| = 65280, the largest bf16
+    value below 2^16: the output must be exactly 2^14 times the unscaled one."""
+    q, k, _ = synth.random_qkv(1, 300, 2, D, synth.BF16, seed=3100 + D)
+    v = _v_in_f16_normal_range(q.shape, 3101 + D)
+    vf = synth.bits_to_float32(v, synth.BF16)
+    v_big = synth.round_to_bits(vf * np.float32(2.0 ** 14), synth.BF16)
+    assert float(np.abs(synth.bits_to_float32(v_big, synth.BF16)).max()) == 65280.0
+    scale = 1.0 / math.sqrt(D)
+    small = run_gpu(q, k, v, scale, synth.BF16)
+    assert_close(small, oracle.attention(q, k, v, scale, synth.BF16), "unscaled")
+    big = run_gpu(q, k, v_big, scale, synth.BF16)
+    assert np.array_equal(big, small * 2.0 ** 14)
+
+
+def test_bf16_v_outside_f16_range_is_reported(cuda_device):
+    import torch
+
+    q, k, v = synth.random_qkv(1, 200, 2, 64, synth.BF16, seed=3102)
+    v = v.copy()
+    v[0, 150, 1, 7] = synth.round_to_bits(np.array([70000.0], np.float32), synth.BF16)[0]
+    tq, tk, tv = (to_dev(x, synth.BF16) for x in (q, k, v))
+    out = torch.empty_like(tq)
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = vitattn.forward_ptr(tq.data_ptr(), tk.data_ptr(), tv.data_ptr(), out.data_ptr(), 1, 200, 2,
+                             64, 0.125, synth.BF16, stream, checked=True)
+    assert rc == -11, vitattn.strerror(rc)
+    # the report does not stick: an in-range call afterwards is clean and right
+    _, _, v_ok = synth.random_qkv(1, 200, 2, 64, synth.BF16, seed=3103)
+    assert_close(run_gpu(q, k, v_ok, 0.125, synth.BF16), oracle.attention(q, k, v_ok, 0.125, synth.BF16))
+
+
+def test_f16_inputs_never_report_range(cuda_device):
+    q, k, v = synth.random_qkv(1, 200, 2, 64, synth.F16, seed=3104)
+    v = synth.round_to_bits(synth.bits_to_float32(v, synth.F16) * np.float32(8192.0), synth.F16)
+    got = run_gpu(q, k, v, 0.125, synth.F16)
+    ref = oracle.attention(q, k, v, 0.125, synth.F16)
+    # relative bar: V is scaled by 2^13
+    assert np.max(np.abs(got - ref)) <= MAX_ABS * 8192.0
+
+
+def test_long_peaky_sequence_full_parity(cuda_device):
+    """The high-resolution recipe (rank-8 logit component of std 4, D = 128) at
+    N = 8192 with 6 heads, every output element against the oracle: long
+    sequences of peaked rows are where the precision of P matters most."""
+    w = synth.Workload("high_res_8k", 1, 8192, 6, 128, synth.BF16, rank8_logit_std=4.0, index=4)
+    q, k, v = synth.make_qkv(w)
+    assert_close(run_gpu(q, k, v, w.scale, w.dtype), oracle.attention(q, k, v, w.scale, w.dtype),
+                 "high_res_8k")

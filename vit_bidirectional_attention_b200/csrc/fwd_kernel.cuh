@@ -6,15 +6,22 @@
 //
 //   S_t   = Q_t K_j^T                    tcgen05.mma, A = Q (smem), B = K (smem), f32 in TMEM
 //   P_t   = exp2(S_t * c - m_t)          softmax warpgroup t, one thread per query row,
-//                                        c = scale*log2(e); P rounded to the input dtype
-//                                        and written back into TMEM over S_t
-//   O_t  += P_t V_j                      tcgen05.mma, A = P (TMEM), B = V (smem), f32 in TMEM
+//                                        c = scale*log2(e); the exponent is rounded to
+//                                        f16 and P = 2^x taken in f16 pairs
+//                                        (ex2.approx.f16x2), written back into TMEM over S_t
+//   O_t  += P_t V_j                      tcgen05.mma, A = P (TMEM), B = V (smem), both f16,
+//                                        f32 in TMEM
 //
 // with the running row maximum m_t, the row sum l_t and the rescaling of O_t
 // kept exact in the online-softmax sense: O and l are always relative to the
 // same (possibly stale) maximum, so the result is O/l at the end.  l_t sums the
-// probabilities after their rounding to the input dtype, i.e. the weights the
-// P.V product really uses.  This is the
+// f16 probabilities themselves, i.e. the weights the P.V product really uses.
+// The P.V product runs in f16 for both input dtypes: f16 has three more
+// mantissa bits than bf16 for P, and its exponential runs at twice the rate
+// of the f32 one.  For bf16 inputs V is converted to f16 in shared memory
+// after it lands (exact for |v| < 2^16 apart from f16's subnormal range,
+// below 2^-14, where the absolute error stays under 2^-25; larger |v| becomes
+// inf and is reported by the checked entry point).  This is the
 // online-softmax GEMM pair of inferencelayer "src/vision_gpu.rs" (doc of
 // `vis_attn_coop_src`: "The obstacle, and the way round it"), except that the
 // running output lives in tensor memory instead of being spilled to shared
@@ -28,7 +35,8 @@
 //   warps 4-7    softmax for query tile 1
 //   warp  8      TMA producer (one lane) and TMEM allocator (whole warp)
 //   warp  9      MMA issuer (one lane)
-//   warps 10-11  idle (they complete the third warpgroup)
+//   warps 10-11  bf16 inputs: convert each V block to f16 in shared memory
+//                (f16 inputs: idle; they complete the third warpgroup)
 // Registers: the launch gives every thread kLaunchRegs; the third warpgroup
 // then gives most of its share back (setmaxnreg.dec to kSideRegs) and the two
 // softmax warpgroups take it (setmaxnreg.inc to kSoftmaxRegs), so a softmax
@@ -64,9 +72,12 @@
 
 #include "ptx.cuh"
 
-// Kernel status word (this header is compiled into exactly one translation
-// unit): 0, or a timeout code from a bounded in-kernel wait.
+// Kernel status words (this header is compiled into exactly one translation
+// unit).  g_vitattn_status: 0, or a timeout code from a bounded in-kernel
+// wait.  g_vitattn_range: nonzero once a bf16 V value of magnitude >= 2^16
+// (outside f16's range) has been converted for the f16 P.V product.
 __device__ unsigned int g_vitattn_status = 0;
+__device__ unsigned int g_vitattn_range = 0;
 
 namespace vitattn {
 
@@ -77,6 +88,7 @@ constexpr int kStages = 4;        // K/V ring slots (K_j, V_j, K_j+1, V_j+1)
 constexpr int kThreads = 384;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kConvWarp = 10;  // first of the two V-converter warps
 // Register split: 3 warps share each SMSP register file (16384 x 32-bit), so a
 // 384-thread block launches at 168 per thread; 2*224 + 56 = 3*168 per SMSP and
 // 256*224 + 128*56 = 384*168 per block: the reallocation never waits forever.
@@ -104,7 +116,8 @@ constexpr int kBarPFull = kBarSFull + kMaxSBufs;
 constexpr int kBarOReady = kBarPFull + 4;            // [2] per tile: a P.V product finished
 constexpr int kBarOFull = kBarOReady + 2;            // [2] per tile: the item's last P.V finished
 constexpr int kBarOEmpty = kBarOFull + 2;            // [2] per tile: the epilogue has read O
-constexpr int kBarDrain = kBarOEmpty + 2;            // [1]
+constexpr int kBarVReady = kBarOEmpty + 2;           // [2] bf16: V block of even / odd index is f16
+constexpr int kBarDrain = kBarVReady + 2;            // [1]
 constexpr int kNumBars = kBarDrain + 1;
 
 // Status codes written to g_vitattn_status (0 = fine).
@@ -303,39 +316,16 @@ __device__ __forceinline__ float row_extreme(const float (&s)[kBlockKeys], int v
     return tree3<kBlockKeys / 32, kNeg>(part);
 }
 
-// Pairs of exponentials (out of every 16 pairs) computed by the polynomial on
-// the FMA/ALU pipes instead of ex2.approx on the MUFU pipe, which runs at 16
-// results per clock per SM and is otherwise the softmax's bottleneck.
-constexpr int kPolyPairs = 0;
-__host__ __device__ constexpr bool poly_pair(int i) { return (i * kPolyPairs) % 16 < kPolyPairs; }
-
-// 2^x for a pair, on the FMA and ALU pipes.  Cody-Waite style split
-// x = j + f with j = round(x) (the 1.5 * 2^23 addition trick leaves j in the
-// low mantissa bits of t) and f in [-1/2, 1/2]; 2^f from a degree-3 minimax
-// polynomial (Remez exchange on the relative error: max 7.5e-5, below the
-// 2^-9 half-ulp of bf16 and about a sixth of an f16 ulp); j is then added to
-// the exponent field.  x is clamped below at -125 so the exponent stays normal.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const float2 magic = make_float2(12582912.f, 12582912.f);
-    const float2 t = ptx::fadd2(x, magic);
-    const float2 f = ptx::fsub2(x, ptx::fsub2(t, magic));
-    float2 p = ptx::ffma2(f, make_float2(0.0551716685f, 0.0551716685f),
-                          make_float2(0.2426111251f, 0.2426111251f));
-    p = ptx::ffma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
-    p = ptx::ffma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
-    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
-// p = 2^(c*s - m) for one block, rounded to the input dtype and written to
-// TMEM as 16-bit pairs at tP (64 columns), 32 scores at a time.  Returns the
-// f32 sum of the ROUNDED p: the tensor core multiplies V by exactly these
-// weights, so normalising by their own sum keeps O a true weighted average of
-// V rows (a single dominant key then gives its V row exactly, whatever the
-// rounding of its weight).
-template <bool kPartial, bool kBF16>
+// p = 2^(c*s - m) for one block in f16, written to TMEM as f16 pairs at tP
+// (64 columns), 32 scores at a time: the exponent x = c*s - m is formed in f32
+// (fma.f32x2), rounded to an f16 pair, and exponentiated by one
+// ex2.approx.f16x2 (maximum relative error about one f16 ulp; subnormal
+// results are kept).  x <= 8 here (the lazy rescale bound), so p <= 256.
+// Returns the f32 sum of these f16 p: the tensor core multiplies V by exactly
+// these weights, so normalising by their own sum keeps O a true weighted
+// average of V rows (a single dominant key then gives its V row exactly,
+// whatever the rounding of its weight).  Columns at or past `valid` get p = 0.
+template <bool kPartial>
 __device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], int valid, float c2,
                                                 float neg_m, uint32_t tP) {
     float acc[4];
@@ -349,25 +339,39 @@ __device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], in
             const int c = 32 * q + 2 * i;
             const float2 x = ptx::ffma2(make_float2(s[c], s[c + 1]), make_float2(c2, c2),
                                         make_float2(neg_m, neg_m));
-            float p0, p1;
-            if (poly_pair(i)) {
-                const float2 e = exp2_poly2(x);
-                p0 = e.x;
-                p1 = e.y;
-            } else {
-                p0 = ptx::ex2(x.x);
-                p1 = ptx::ex2(x.y);
-            }
-            if (kPartial) {
-                p0 = c < valid ? p0 : 0.f;
-                p1 = c + 1 < valid ? p1 : 0.f;
-            }
-            pk[i] = ptx::pack2<kBF16>(p0, p1);
-            ptx::add_halves<kBF16>(pk[i], acc[2 * (i & 1)], acc[2 * (i & 1) + 1]);
+            pk[i] = ptx::ex2_h2(ptx::pack2<false>(x.x, x.y));
+            if (kPartial)
+                pk[i] &= (c < valid ? 0x0000FFFFu : 0u) | (c + 1 < valid ? 0xFFFF0000u : 0u);
+            ptx::add_halves<false>(pk[i], acc[2 * (i & 1)], acc[2 * (i & 1) + 1]);
         }
         ptx::tmem_st16(tP + 16 * q, pk);
     }
     return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// One V block (a 128 x DP tile, 16-bit elements, any swizzle: the conversion
+// is elementwise and in place) from bf16 to f16, by the 64 threads of the two
+// converter warps; ct is the thread's index among them.  Returns the largest
+// |v| seen, so that values outside f16's range can be reported.
+template <int TILE>
+__device__ __forceinline__ float convert_v_tile(uint8_t* tile, int ct, float vmax) {
+    constexpr int NV = TILE / 16 / 64;  // 16-byte vectors per thread
+    static_assert(TILE % (16 * 64) == 0, "converter split");
+    uint4* const v = reinterpret_cast<uint4*>(tile);
+#pragma unroll 4
+    for (int i = 0; i < NV; ++i) {
+        uint4 w = v[ct + 64 * i];
+        uint32_t* const u = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(u[e] << 16);
+            const float hi = __uint_as_float(u[e] & 0xFFFF0000u);
+            vmax = ptx::fmax3(vmax, fabsf(lo), fabsf(hi));
+            u[e] = ptx::pack2<false>(lo, hi);
+        }
+        v[ct + 64 * i] = w;
+    }
+    return vmax;
 }
 
 // Multiply this thread's row of O (DP columns of TMEM at tO) by alpha.
@@ -496,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             ptx::mbar_init(bar(kBarOReady + t), 1);
             ptx::mbar_init(bar(kBarOFull + t), 1);
             ptx::mbar_init(bar(kBarOEmpty + t), 4 * 32);
+            ptx::mbar_init(bar(kBarVReady + t), 2 * 32);
         }
         ptx::mbar_init(bar(kBarDrain), 1);
         *abort_flag = 0;
@@ -583,7 +588,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the issue loop (its control flow and descriptors
+        // stay warp-uniform); one elected lane issues each MMA and commit.
+        {
+            const uint32_t leader = ptx::elect_one();
             // Descriptors are built once per chunk and phase; a K step then
             // only adds a constant to the start-address field (16-byte units),
             // so the single issuing thread spends its time issuing MMAs.
@@ -601,11 +609,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                                               16u * (uint32_t)w, swizzle_code(w));
 #pragma unroll
                     for (int kk = 0; kk < w / 16; ++kk)
-                        ptx::mma_ss(d, qd + 2u * kk, kd + 2u * kk, idS,
-                                    (c == 0 && kk == 0) ? 0u : 1u);
+                        ptx::mma_ss_w(d, qd + 2u * kk, kd + 2u * kk, idS,
+                                      (c == 0 && kk == 0) ? 0u : 1u, leader);
                 }
             };
-            // P.V: the 64-column chunks of V form one MMA with N = 64 * n64 (the
+            // P.V (f16 x f16): the 64-column chunks of V form one MMA with N = 64 * n64 (the
             // second 64-column swizzle atom sits one chunk, 16 KB, further: the
             // leading byte offset); narrower tail chunks get an MMA each.
             constexpr int N64 = DP / 64;
@@ -627,14 +635,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 for (int ks = 0; ks < kBlockKeys / 16; ++ks) {
                     const uint32_t acc = (accumulate || ks > 0) ? 1u : 0u;
                     if (N64 > 0)
-                        ptx::mma_ts(d, a + (uint32_t)(ks * 8), vd64 + (uint64_t)(2 * 64 * ks),
-                                    idesc_f16(kBF16, 64 * N64, true), acc);
+                        ptx::mma_ts_w(d, a + (uint32_t)(ks * 8), vd64 + (uint64_t)(2 * 64 * ks),
+                                      idesc_f16(false, 64 * N64, true), acc, leader);
 #pragma unroll
                     for (int i = 0; i < NTAIL; ++i) {
                         const int c = N64 + i;
                         const int w = chunk_width(DP, c);
-                        ptx::mma_ts(d + (uint32_t)chunk_col(DP, c), a + (uint32_t)(ks * 8),
-                                    vdt[i] + (uint64_t)(2 * w * ks), idesc_f16(kBF16, w, true), acc);
+                        ptx::mma_ts_w(d + (uint32_t)chunk_col(DP, c), a + (uint32_t)(ks * 8),
+                                      vdt[i] + (uint64_t)(2 * w * ks), idesc_f16(false, w, true), acc, leader);
                     }
                 }
             };
@@ -665,39 +673,44 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             auto issue_s = [&](const Cursor& c) -> bool {
                 const int qb = c.k % NQ;
                 if (c.j == 0) {  // first S of this tile in this item: its Q tile
-                    if (!wait_one(bar(kBarQFull + 2 * qb + c.t), (uint32_t)(c.k / NQ) & 1u, abort_flag, tmo, 2))
+                    if (!wait_warp(bar(kBarQFull + 2 * qb + c.t), (uint32_t)(c.k / NQ) & 1u, abort_flag, tmo, 2))
                         return false;
                     ptx::tc_fence_after();
                 }
                 if (c.t == 0) {
-                    if (!wait_one(bar(kBarKvFull + kv_slot(2 * c.g)), kv_parity(2 * c.g), abort_flag, tmo, 3))
+                    if (!wait_warp(bar(kBarKvFull + kv_slot(2 * c.g)), kv_parity(2 * c.g), abort_flag, tmo, 3))
                         return false;
                     ptx::tc_fence_after();
                 }
                 mma_s(qb * kTilesPerCta + c.t, kv_slot(2 * c.g), c.buf);
-                ptx::mma_commit(bar(kBarSFull + c.buf));
-                if (c.t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * c.g)));
-                if (kLoop && c.j == nkb - 1) ptx::mma_commit(bar(kBarQEmpty + 2 * qb + c.t));
+                ptx::mma_commit_w(bar(kBarSFull + c.buf), leader);
+                if (c.t == T - 1) ptx::mma_commit_w(bar(kBarKvEmpty + kv_slot(2 * c.g)), leader);
+                if (kLoop && c.j == nkb - 1) ptx::mma_commit_w(bar(kBarQEmpty + 2 * qb + c.t), leader);
                 return true;
             };
-            // O_t += P V_j; V_j is waited for by its first unit and released after its last.
+            // O_t += P V_j; V_j is waited for by its first unit (landed, and for
+            // bf16 inputs converted to f16) and released after its last.  The
+            // converter is at most two blocks ahead (it needs V_j+2's slot, which
+            // the last P.V of block j frees), so the parity of V-ready is unambiguous.
             auto issue_pv = [&](const Cursor& c) -> bool {
                 const int t = c.t, j = c.j, g = c.g;
                 if (t == 0 &&
-                    !wait_one(bar(kBarKvFull + kv_slot(2 * g + 1)), kv_parity(2 * g + 1), abort_flag, tmo, 4))
+                    !(kBF16 ? wait_warp(bar(kBarVReady + (g & 1)), (uint32_t)(g >> 1) & 1u, abort_flag, tmo, 4)
+                            : wait_warp(bar(kBarKvFull + kv_slot(2 * g + 1)), kv_parity(2 * g + 1), abort_flag,
+                                       tmo, 4)))
                     return false;
                 // the first product of an item overwrites O_t: the previous item's
                 // epilogue must have read it out
                 if (kLoop && j == 0 && c.k > 0 &&
-                    !wait_one(bar(kBarOEmpty + t), (uint32_t)(c.k - 1) & 1u, abort_flag, tmo, 13))
+                    !wait_warp(bar(kBarOEmpty + t), (uint32_t)(c.k - 1) & 1u, abort_flag, tmo, 13))
                     return false;
-                if (!wait_one(bar(kBarPFull + 2 * t + (g & 1)), (uint32_t)(g >> 1) & 1u, abort_flag, tmo, 5))
+                if (!wait_warp(bar(kBarPFull + 2 * t + (g & 1)), (uint32_t)(g >> 1) & 1u, abort_flag, tmo, 5))
                     return false;
                 ptx::tc_fence_after();
                 mma_pv(t, kv_slot(2 * g + 1), c.buf, j > 0);
-                if (track_pv) ptx::mma_commit(bar(kBarOReady + t));
-                if (t == T - 1) ptx::mma_commit(bar(kBarKvEmpty + kv_slot(2 * g + 1)));
-                if (j == nkb - 1) ptx::mma_commit(bar(kBarOFull + t));
+                if (track_pv) ptx::mma_commit_w(bar(kBarOReady + t), leader);
+                if (t == T - 1) ptx::mma_commit_w(bar(kBarKvEmpty + kv_slot(2 * g + 1)), leader);
+                if (j == nkb - 1) ptx::mma_commit_w(bar(kBarOFull + t), leader);
                 return true;
             };
 
@@ -720,11 +733,28 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             }
             if (!ok) {
                 // every MMA issued so far must finish before TMEM is freed
-                ptx::mma_commit(bar(kBarDrain));
+                ptx::mma_commit_w(bar(kBarDrain), leader);
                 wait_drain(bar(kBarDrain), 0, 200000000ull);
             }
         }
         __syncwarp();
+    } else if (kBF16) {
+        // ------------------------------------------------------------ V converter (bf16)
+        // V_g (ring entry 2g+1) is converted in place once it lands; both
+        // warps then signal V-ready for it (64 arrivals).
+        const int ct = threadIdx.x - kConvWarp * 32;
+        const int nblocks = n_my * nkb;
+        float vmax = 0.f;
+        for (int g = 0; g < nblocks; ++g) {
+            const int idx = 2 * g + 1;
+            const int slot = idx % kStages;
+            if (!wait_warp(bar(kBarKvFull + slot), (uint32_t)(idx / kStages) & 1u, abort_flag, tmo, 14))
+                break;
+            vmax = convert_v_tile<TILE>(base_ptr + (sKV - base) + slot * TILE, ct, vmax);
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(bar(kBarVReady + (g & 1)));
+        }
+        if (vmax >= 65536.f) atomicOr(&g_vitattn_range, 1u);
     }
     } else {
         ptx::setmaxnreg_inc<kSoftmaxRegs>();
@@ -789,8 +819,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     m_used = m_new;
                     l *= alpha;
                 }
-                l += partial ? exp_pack_store<true, kBF16>(s, valid, c2, -m_used, tS)
-                             : exp_pack_store<false, kBF16>(s, valid, c2, -m_used, tS);
+                l += partial ? exp_pack_store<true>(s, valid, c2, -m_used, tS)
+                             : exp_pack_store<false>(s, valid, c2, -m_used, tS);
                 // Bring O_t (P.V up to block j-1) to the new reference maximum before
                 // P_t,j.V_j is issued.  The product of block j-1 may still be running:
                 // wait for it (phase j-1 of the per-tile "P.V done" barrier; the phase

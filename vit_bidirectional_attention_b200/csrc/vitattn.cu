@@ -243,14 +243,20 @@ int forward_checked(const void* q, const void* k, const void* v, void* out, int6
     cudaError_t e = cudaMemcpyToSymbolAsync(g_vitattn_status, &zero, sizeof zero, 0,
                                             cudaMemcpyHostToDevice, stream);
     if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemcpyToSymbolAsync(g_vitattn_range, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,
+                                stream);
+    if (e != cudaSuccess) return cuda_fail(e);
     rc = launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags);
     if (rc) return rc;
     e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    unsigned status = 0;
+    unsigned status = 0, range = 0;
     e = cudaMemcpyFromSymbol(&status, g_vitattn_status, sizeof status);
     if (e != cudaSuccess) return cuda_fail(e);
-    return status ? VITATTN_ERR_TIMEOUT : VITATTN_OK;
+    e = cudaMemcpyFromSymbol(&range, g_vitattn_range, sizeof range);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (status) return VITATTN_ERR_TIMEOUT;
+    return range ? VITATTN_ERR_RANGE : VITATTN_OK;
 }
 
 }  // namespace
@@ -320,6 +326,7 @@ const char* vitattn_strerror(int status) {
         case VITATTN_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
         case VITATTN_ERR_SCALE: return "scale must be finite";
         case VITATTN_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+        case VITATTN_ERR_RANGE: return "a bf16 V value has magnitude >= 65536, outside the f16 P.V product's range";
         default: return "unknown status";
     }
 }

@@ -26,6 +26,7 @@ STATUS_NAMES = {
     -8: "VITATTN_ERR_TIMEOUT",
     -9: "VITATTN_ERR_SCALE",
     -10: "VITATTN_ERR_DEVICE",
+    -11: "VITATTN_ERR_RANGE",
 }
 
 _lib = None
