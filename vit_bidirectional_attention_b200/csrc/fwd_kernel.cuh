@@ -6,9 +6,8 @@
 //
 //   S_t   = Q_t K_j^T                    tcgen05.mma, A = Q (smem), B = K (smem), f32 in TMEM
 //   P_t   = exp2(S_t * c - m_t)          softmax warpgroup t, one thread per query row,
-//                                        c = scale*log2(e); the exponent is rounded to
-//                                        f16 and P = 2^x taken in f16 pairs
-//                                        (ex2.approx.f16x2), written back into TMEM over S_t
+//                                        c = scale*log2(e); P rounded to f16 and written
+//                                        back into TMEM over S_t
 //   O_t  += P_t V_j                      tcgen05.mma, A = P (TMEM), B = V (smem), both f16,
 //                                        f32 in TMEM
 //
@@ -17,8 +16,7 @@
 // same (possibly stale) maximum, so the result is O/l at the end.  l_t sums the
 // f16 probabilities themselves, i.e. the weights the P.V product really uses.
 // The P.V product runs in f16 for both input dtypes: f16 has three more
-// mantissa bits than bf16 for P, and its exponential runs at twice the rate
-// of the f32 one.  For bf16 inputs V is converted to f16 in shared memory
+// mantissa bits than bf16 for P.  For bf16 inputs V is converted to f16 in shared memory
 // after it lands (exact for |v| < 2^16 apart from f16's subnormal range,
 // below 2^-14, where the absolute error stays under 2^-25; larger |v| becomes
 // inf and is reported by the checked entry point).  This is the
@@ -316,15 +314,41 @@ __device__ __forceinline__ float row_extreme(const float (&s)[kBlockKeys], int v
     return tree3<kBlockKeys / 32, kNeg>(part);
 }
 
-// p = 2^(c*s - m) for one block in f16, written to TMEM as f16 pairs at tP
-// (64 columns), 32 scores at a time: the exponent x = c*s - m is formed in f32
-// (fma.f32x2), rounded to an f16 pair, and exponentiated by one
-// ex2.approx.f16x2 (maximum relative error about one f16 ulp; subnormal
-// results are kept).  x <= 8 here (the lazy rescale bound), so p <= 256.
-// Returns the f32 sum of these f16 p: the tensor core multiplies V by exactly
-// these weights, so normalising by their own sum keeps O a true weighted
-// average of V rows (a single dominant key then gives its V row exactly,
-// whatever the rounding of its weight).  Columns at or past `valid` get p = 0.
+// Pairs of exponentials (out of every 16 pairs) computed by the polynomial on
+// the FMA/ALU pipes instead of ex2.approx on the MUFU pipe, which runs at 16
+// results per clock per SM (f32 and f16 pairs alike, measured in the softmax
+// loop) and is otherwise the softmax's bottleneck.
+constexpr int kPolyPairs = 0;
+__host__ __device__ constexpr bool poly_pair(int i) { return (i * kPolyPairs) % 16 < kPolyPairs; }
+
+// 2^x for a pair, on the FMA and ALU pipes.  Cody-Waite style split
+// x = j + f with j = round(x) (adding 1.5 * 2^23 leaves j in the low mantissa
+// bits of t) and f in [-1/2, 1/2]; 2^f from a degree-3 minimax polynomial
+// (Remez exchange on the relative error: max 7.5e-5, about a sixth of an f16
+// ulp); j is then added to the exponent field.  x is clamped below at -125 so
+// the exponent stays normal (such p round to 0 in f16 anyway).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    const float2 t = ptx::fadd2(x, magic);
+    const float2 f = ptx::fsub2(x, ptx::fsub2(t, magic));
+    float2 p = ptx::ffma2(f, make_float2(0.0551716685f, 0.0551716685f),
+                          make_float2(0.2426111251f, 0.2426111251f));
+    p = ptx::ffma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
+    p = ptx::ffma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// p = 2^(c*s - m) for one block, in f32 (ex2.approx, or the polynomial for
+// some pairs), rounded to f16 and written to TMEM as f16 pairs at tP (64
+// columns), 32 scores at a time.  x <= 8 here (the lazy rescale bound), so
+// p <= 256; f16 keeps p down to 2^-24 (subnormals are kept).  Returns the f32
+// sum of the ROUNDED p: the tensor core multiplies V by exactly these
+// weights, so normalising by their own sum keeps O a true weighted average of
+// V rows (a single dominant key then gives its V row exactly, whatever the
+// rounding of its weight).  Columns at or past `valid` get p = 0.
 template <bool kPartial>
 __device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], int valid, float c2,
                                                 float neg_m, uint32_t tP) {
@@ -339,9 +363,20 @@ __device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], in
             const int c = 32 * q + 2 * i;
             const float2 x = ptx::ffma2(make_float2(s[c], s[c + 1]), make_float2(c2, c2),
                                         make_float2(neg_m, neg_m));
-            pk[i] = ptx::ex2_h2(ptx::pack2<false>(x.x, x.y));
-            if (kPartial)
-                pk[i] &= (c < valid ? 0x0000FFFFu : 0u) | (c + 1 < valid ? 0xFFFF0000u : 0u);
+            float p0, p1;
+            if (poly_pair(i)) {
+                const float2 e = exp2_poly2(x);
+                p0 = e.x;
+                p1 = e.y;
+            } else {
+                p0 = ptx::ex2(x.x);
+                p1 = ptx::ex2(x.y);
+            }
+            if (kPartial) {
+                p0 = c < valid ? p0 : 0.f;
+                p1 = c + 1 < valid ? p1 : 0.f;
+            }
+            pk[i] = ptx::pack2<false>(p0, p1);
             ptx::add_halves<false>(pk[i], acc[2 * (i & 1)], acc[2 * (i & 1) + 1]);
         }
         ptx::tmem_st16(tP + 16 * q, pk);

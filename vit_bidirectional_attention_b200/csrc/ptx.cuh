@@ -299,14 +299,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x for both f16 halves of a word (MUFU: one instruction for two results).
-// Subnormal results are kept, not flushed.
-__device__ __forceinline__ uint32_t ex2_h2(uint32_t x) {
-    uint32_t y;
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
-
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (TMA, tcgen05.mma operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
