@@ -115,6 +115,28 @@ def probs(q, k, scale: float, dtype: int, b: int, h: int) -> np.ndarray:
     return P
 
 
+def attention_varlen(q, k, v, cu_seqlens, scale: float, dtype: int, mode: int = MODE_TWO_PASS) -> np.ndarray:
+    """Ragged batch of images packed along the token axis: ``q, k, v`` are
+    ``[total, H, D]`` and segment s covers tokens ``cu_seqlens[s] ..
+    cu_seqlens[s+1] - 1``.  Each token attends to the keys of its own segment
+    only, so every segment is an independent attention problem
+    (inferencelayer ``src/vision_gpu.rs``, the vision tower's ``forward``:
+    attention over an image is one ragged segment given by its start
+    offsets, and several images are several segments).  Returns
+    ``[total, H, D]`` float64; tokens of no segment (none, for valid offsets)
+    stay zero."""
+    cu = [int(x) for x in cu_seqlens]
+    if len(cu) < 2 or cu[0] != 0 or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must start at 0 and be nondecreasing")
+    if cu[-1] != q.shape[0]:
+        raise ValueError("cu_seqlens must end at the token count")
+    out = np.zeros(q.shape, np.float64)
+    for a, b in zip(cu, cu[1:]):
+        if b > a:
+            out[a:b] = attention(q[None, a:b], k[None, a:b], v[None, a:b], scale, dtype, mode)[0]
+    return out
+
+
 def widen(bits: np.ndarray, dtype: int) -> np.ndarray:
     """bf16 / f16 bit patterns to float64, exactly."""
     bits = np.ascontiguousarray(bits, dtype=np.uint16)

@@ -302,3 +302,60 @@ def test_rank8_recipe_reaches_logit_std_4():
     qf, kf = (synth.bits_to_float32(x, synth.BF16).astype(np.float64) for x in (q, k))
     s = np.einsum("nd,md->nm", qf[0, :, 0], kf[0, :, 0]) / math.sqrt(128)
     assert 3.6 < s.std() < 4.4
+
+
+# ---------------------------------------------------------------- ragged (multi-image) batches
+
+def _block_diag_brute(qf, kf, vf, cu, scale):
+    """Independent formulation: one softmax over the whole packed token axis
+    with every key outside the query's own segment masked to -inf."""
+    T, H, D = qf.shape
+    seg = np.zeros(T, np.int64)
+    for s, (a, b) in enumerate(zip(cu, cu[1:])):
+        seg[a:b] = s
+    out = np.zeros((T, H, D))
+    for h in range(H):
+        logits = scale * (qf[:, h, :] @ kf[:, h, :].T)
+        logits[seg[:, None] != seg[None, :]] = -np.inf
+        logits -= logits.max(axis=1, keepdims=True)
+        w = np.exp(logits)
+        w /= w.sum(axis=1, keepdims=True)
+        out[:, h, :] = w @ vf[:, h, :]
+    return out
+
+
+@pytest.mark.parametrize("cu", [[0, 5], [0, 1, 4, 9], [0, 3, 3, 7, 8], [0, 0, 6, 6, 13]])
+def test_varlen_oracle_matches_block_diagonal_masked_softmax(cu):
+    T, H, D = cu[-1], 2, 8
+    q, k, v = (synth.round_to_bits(rnd((T, H, D), 90 + i, 1.5).astype(np.float32), synth.BF16) for i in range(3))
+    got = oracle.attention_varlen(q, k, v, cu, 0.4, oracle.BF16)
+    qf, kf, vf = (oracle.widen(x, oracle.BF16) for x in (q, k, v))
+    np.testing.assert_allclose(got, _block_diag_brute(qf, kf, vf, cu, 0.4), rtol=0, atol=1e-12)
+
+
+def test_varlen_oracle_equal_segments_is_the_dense_batch():
+    B, N, H, D = 3, 7, 2, 16
+    q, k, v = synth.random_qkv(B, N, H, D, synth.F16, seed=91)
+    dense = oracle.attention(q, k, v, 0.25, oracle.F16)
+    packed = oracle.attention_varlen(q.reshape(B * N, H, D), k.reshape(B * N, H, D), v.reshape(B * N, H, D),
+                                     [0, N, 2 * N, 3 * N], 0.25, oracle.F16)
+    assert np.array_equal(packed.reshape(B, N, H, D), dense)
+
+
+def test_varlen_oracle_segments_do_not_see_each_other():
+    cu = [0, 4, 10]
+    q, k, v = (synth.round_to_bits(rnd((10, 2, 8), 92 + i).astype(np.float32), synth.BF16) for i in range(3))
+    a = oracle.attention_varlen(q, k, v, cu, 0.5, oracle.BF16)
+    k2, v2 = k.copy(), v.copy()
+    k2[4:] = synth.round_to_bits(rnd((6, 2, 8), 95).astype(np.float32), synth.BF16)
+    v2[4:] = synth.round_to_bits(rnd((6, 2, 8), 96).astype(np.float32), synth.BF16)
+    b = oracle.attention_varlen(q, k2, v2, cu, 0.5, oracle.BF16)
+    assert np.array_equal(a[:4], b[:4])
+    assert not np.array_equal(a[4:], b[4:])
+
+
+def test_varlen_oracle_rejects_bad_offsets():
+    q = np.zeros((4, 1, 8), np.uint16)
+    for cu in ([1, 4], [0, 3, 2, 4], [0, 3]):
+        with pytest.raises(ValueError):
+            oracle.attention_varlen(q, q, q, cu, 1.0, oracle.BF16)
