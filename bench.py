@@ -3,6 +3,9 @@
 
 A step is one call of ``vitattn_forward`` over one batch of the workload:
 the whole path (Q.K^T, online softmax, P.V, epilogue) in one kernel launch.
+For a ragged multi-image workload (``--workload multi_image``) a step is one
+call of ``vitattn_forward_varlen`` over the packed batch, and the flops are
+4*H*D*sum(n_s^2) over its images.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
@@ -10,7 +13,9 @@ the whole path (Q.K^T, online softmax, P.V, epilogue) in one kernel launch.
   timed region (CUDA events on the launching stream, max over ranks), TFLOP/s.
 * ``e2e``: the same metric through the host-buffer entry point
   ``vitattn_forward_host`` (pinned host -> device copies of q, k, v, the
-  kernel, device -> host copy of out, all inside the timed region).
+  kernel, device -> host copy of out, all inside the timed region); for a
+  ragged workload through the Python entry ``forward_varlen`` with the same
+  copies issued on the same stream.
 * ``roofline``: the kernel against the measured dense bf16 tensor peak.
 * ``cpu_baseline``: the fp64 oracle on this host's cores, on a bounded sample
   of output rows of the same workload, scaled to the same metric.
@@ -36,6 +41,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
+
 from vit_bidirectional_attention_b200 import ranks, synth  # noqa: E402
 
 DEFAULT_WORKLOAD = "batched"
@@ -53,7 +60,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=None,
                     help="timed steps (default: enough for about 2 s of timed work)")
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS) + sorted(synth.RAGGED))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -158,22 +165,44 @@ class ClockSampler:
                 "reasons": sorted(active), "samples": len(loaded), "window": window}
 
 
+def oracle_rows(w, q, k, v, rows):
+    """The oracle on sampled output rows; returns the flops those rows cost."""
+    import oracle
+
+    if isinstance(w, synth.RaggedWorkload):
+        oracle.attention_varlen_rows(q, k, v, w.cu_seqlens, w.scale, w.dtype, rows)
+        seg_len = np.diff(np.asarray(w.cu_seqlens))
+        tok_seg = np.repeat(np.arange(len(seg_len)), seg_len)
+        return float(4.0 * w.D * seg_len[tok_seg[np.asarray(rows) // w.H]].sum())
+    oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
+    return 4.0 * w.N * w.D * len(rows)
+
+
+def total_rows_of(w):
+    return (w.total if isinstance(w, synth.RaggedWorkload) else w.B * w.N) * w.H
+
+
+def sample_rows_of(w, count, seed):
+    if isinstance(w, synth.RaggedWorkload):
+        return synth.sample_rows((1, w.total, w.H), count, seed)
+    return synth.sample_rows(w, count, seed)
+
+
 def cpu_baseline(w, q, k, v, seconds: float):
     """The fp64 oracle, as it stands, on a bounded sample of output rows."""
     import oracle
 
-    flops_per_row = 4.0 * w.N * w.D
-    total_rows = w.B * w.N * w.H
+    total_rows = total_rows_of(w)
     n = min(64, total_rows)
     for attempt in range(6):
-        rows = synth.sample_rows(w, n, seed=w.seed + 11 + attempt)
+        rows = sample_rows_of(w, n, seed=w.seed + 11 + attempt)
         t0 = time.perf_counter()
-        oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
+        flops = oracle_rows(w, q, k, v, rows)
         dt = time.perf_counter() - t0
         if dt >= 0.5 * seconds or len(rows) >= total_rows:
             break
         n = int(min(total_rows, max(2 * n, len(rows) * seconds / max(dt, 1e-6))))
-    return {"value": flops_per_row * len(rows) / dt / 1e12, "unit": "TFLOP/s",
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{len(rows)} of {total_rows} output rows (seeded), fp64, "
                       f"{dt:.1f} s on {oracle.num_threads()} threads"}
@@ -199,6 +228,22 @@ def max_over_ranks(x: float, world: int) -> float:
     return ranks.max_over_ranks(x, world, device="cuda")
 
 
+def load_workload(name):
+    """(workload, q, k, v): dense [B, N, H, D] or ragged [total, H, D] bit arrays."""
+    if name in synth.RAGGED:
+        w = synth.RAGGED[name]
+        return (w,) + tuple(synth.make_qkv_ragged(w))
+    w = synth.WORKLOADS[name]
+    return (w,) + tuple(synth.make_qkv(w))
+
+
+def shape_config(w):
+    if isinstance(w, synth.RaggedWorkload):
+        return {"images": len(w.seqlens), "seqlens": list(w.seqlens), "total_tokens": w.total,
+                "H": w.H, "D": w.D}
+    return {"B": w.B, "N": w.N, "H": w.H, "D": w.D}
+
+
 def run_reference(args):
     """The oracle as the reference arm: bounded samples on the host cores."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -207,35 +252,33 @@ def run_reference(args):
         return 0
     import oracle
 
-    w = synth.WORKLOADS[args.workload]
-    q, k, v = synth.make_qkv(w)
+    w, q, k, v = load_workload(args.workload)
     if args.steps is None:
         args.steps = 5
-    total_rows = w.B * w.N * w.H
+    total_rows = total_rows_of(w)
     per_step = max(1.0, min(2.0, 120.0 / max(1, args.steps + args.warmup)))
-    rows_probe = synth.sample_rows(w, min(64, total_rows), seed=w.seed + 17)
+    rows_probe = sample_rows_of(w, min(64, total_rows), seed=w.seed + 17)
     t0 = time.perf_counter()
-    oracle.attention_rows(q, k, v, w.scale, w.dtype, rows_probe)
+    oracle_rows(w, q, k, v, rows_probe)
     t_probe = max(time.perf_counter() - t0, 1e-6)
     n_rows = int(min(total_rows, max(32, len(rows_probe) * per_step / t_probe)))
-    flops_per_row = 4.0 * w.N * w.D
-    times = []
+    times, flops = [], []
     for i in range(args.warmup + args.steps):
-        rows = synth.sample_rows(w, n_rows, seed=w.seed + 1000 + i)
+        rows = sample_rows_of(w, n_rows, seed=w.seed + 1000 + i)
         t0 = time.perf_counter()
-        oracle.attention_rows(q, k, v, w.scale, w.dtype, rows)
+        f = oracle_rows(w, q, k, v, rows)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
+            flops.append(f)
     step_s = sum(times) / len(times)
-    value = flops_per_row * n_rows / step_s / 1e12
+    value = sum(flops) / sum(times) / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "B": w.B, "N": w.N, "H": w.H, "D": w.D,
-                   "input_dtype": synth.DTYPE_NAMES[w.dtype], "scale": w.scale,
-                   "sample_rows_per_step": n_rows},
+        "config": dict(shape_config(w), workload=args.workload, input_dtype=synth.DTYPE_NAMES[w.dtype],
+                       scale=w.scale, sample_rows_per_step=n_rows),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle",
                          "sample": f"{n_rows} of {total_rows} output rows per step (seeded)"},
@@ -255,8 +298,8 @@ def main():
     from vit_bidirectional_attention_b200 import vitattn
 
     world, rank, local = dist_setup(args)
-    w = synth.WORKLOADS[args.workload]
-    q, k, v = synth.make_qkv(w)
+    w, q, k, v = load_workload(args.workload)
+    ragged = isinstance(w, synth.RaggedWorkload)
     tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
     dev = torch.device("cuda", local if world > 1 else 0)
 
@@ -270,18 +313,34 @@ def main():
     sh = stream.cuda_stream
     L = vitattn.lib()
 
-    def step():
-        rc = L.vitattn_forward(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
-                               w.N, w.H, w.D, w.scale, w.dtype, sh)
-        if rc:
-            raise vitattn.VitAttnError(rc, "vitattn_forward")
+    if ragged:
+        import ctypes
+
+        cu_arr = (ctypes.c_int32 * len(w.cu_seqlens))(*w.cu_seqlens)
+        cu_ptr, n_seqs = ctypes.cast(cu_arr, ctypes.c_void_p), len(w.seqlens)
+
+        def step():
+            rc = L.vitattn_forward_varlen(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), cu_ptr,
+                                          n_seqs, w.H, w.D, w.scale, w.dtype, sh)
+            if rc:
+                raise vitattn.VitAttnError(rc, "vitattn_forward_varlen")
+    else:
+        def step():
+            rc = L.vitattn_forward(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
+                                   w.N, w.H, w.D, w.scale, w.dtype, sh)
+            if rc:
+                raise vitattn.VitAttnError(rc, "vitattn_forward")
 
     # correctness gate on this exact launch configuration before timing
     with torch.cuda.stream(stream):
-        rc = vitattn.forward_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
-                                 w.N, w.H, w.D, w.scale, w.dtype, sh, checked=True)
+        if ragged:
+            rc = vitattn.forward_varlen_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(),
+                                            w.cu_seqlens, w.H, w.D, w.scale, w.dtype, sh, checked=True)
+        else:
+            rc = vitattn.forward_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
+                                     w.N, w.H, w.D, w.scale, w.dtype, sh, checked=True)
     if rc:
-        raise vitattn.VitAttnError(rc, "vitattn_forward_checked")
+        raise vitattn.VitAttnError(rc, "checked forward")
 
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     sampler.start()
@@ -330,22 +389,31 @@ def main():
     hout_p = torch.empty_like(hq).pin_memory()
     e2e_steps = max(1, args.e2e_steps)
 
-    def e2e_step():
-        rc = L.vitattn_forward_host(hq_p.data_ptr(), hk_p.data_ptr(), hv_p.data_ptr(),
-                                    hout_p.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                                    dout.data_ptr(), w.B, w.N, w.H, w.D, w.scale, w.dtype, sh)
-        if rc:
-            raise vitattn.VitAttnError(rc, "vitattn_forward_host")
+    if ragged:
+        def e2e_step():
+            for d, h in ((dq, hq_p), (dk, hk_p), (dv, hv_p)):
+                d.copy_(h, non_blocking=True)
+            vitattn.forward_varlen(dq, dk, dv, w.cu_seqlens, out=dout, scale=w.scale, stream=stream)
+            hout_p.copy_(dout, non_blocking=True)
+    else:
+        def e2e_step():
+            rc = L.vitattn_forward_host(hq_p.data_ptr(), hk_p.data_ptr(), hv_p.data_ptr(),
+                                        hout_p.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                        dout.data_ptr(), w.B, w.N, w.H, w.D, w.scale, w.dtype, sh)
+            if rc:
+                raise vitattn.VitAttnError(rc, "vitattn_forward_host")
 
-    for _ in range(2):
-        e2e_step()
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            e2e_step()
     stream.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
     e1.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
@@ -378,15 +446,15 @@ def main():
             "vs_baseline": None,
             "dtype": synth.DTYPE_NAMES[w.dtype],
             "data": "synthetic (seeded normals with the workload's shape and distribution)",
-            "config": {
-                "workload": args.workload, "B": w.B, "N": w.N, "H": w.H, "D": w.D,
-                "scale": w.scale, "global_batch": w.B * world,
-                "parallelism": f"independent (b,h) units per GPU x{world}",
+            "config": dict(shape_config(w), **{
+                "workload": args.workload,
+                "scale": w.scale, "global_batch": (len(w.seqlens) if ragged else w.B) * world,
+                "parallelism": f"independent ({'image' if ragged else 'b'},h) units per GPU x{world}",
                 "l2": (f"inputs {w.io_bytes / 2**20:.0f} MiB > 126 MiB L2, no flush"
                        if w.io_bytes > L2_BYTES else
                        f"inputs {w.io_bytes / 2**20:.1f} MiB fit in L2 (warm)"),
                 "flops_per_step": w.flops,
-            },
+            }),
             "pct_of_datasheet_peak": 100.0 * per_gpu_tflops / DATASHEET_PEAK_TFLOPS,
             "roofline": {
                 "bound": "tensor",
@@ -403,7 +471,8 @@ def main():
             },
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": 3 * w.numel * 2, "d2h_bytes_per_step": w.numel * 2,
-                    "ms_per_step": e2e_ms / e2e_steps, "entry": "vitattn_forward_host"},
+                    "ms_per_step": e2e_ms / e2e_steps,
+                    "entry": "forward_varlen + stream copies" if ragged else "vitattn_forward_host"},
             "gpu_launches": args.steps * vitattn.launches_per_call(),
             "clocks": clocks,
             "cpu_baseline": cpu,

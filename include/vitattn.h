@@ -84,7 +84,8 @@ enum vitattn_status {
     VITATTN_ERR_TIMEOUT = -8, /* a bounded in-kernel wait ran out (checked entry only) */
     VITATTN_ERR_SCALE = -9,   /* scale is NaN or infinite */
     VITATTN_ERR_DEVICE = -10, /* the current device is not an sm_100 GPU */
-    VITATTN_ERR_RANGE = -11   /* a bf16 V value has |v| >= 65536 (checked entry only) */
+    VITATTN_ERR_RANGE = -11,  /* a bf16 V value has |v| >= 65536 (checked entry only) */
+    VITATTN_ERR_SEQLENS = -12 /* cu_seqlens does not start at 0 or decreases somewhere */
 };
 
 /*
@@ -114,6 +115,49 @@ VITATTN_API int vitattn_forward(const void* q, const void* k, const void* v, voi
 VITATTN_API int vitattn_forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B,
                             int64_t N, int64_t H, int64_t D, float scale, int dtype,
                             vitattn_stream_t stream);
+
+/* Most segments one vitattn_forward_varlen call takes. */
+#define VITATTN_MAX_SEQS 256
+
+/*
+ * vitattn_forward_varlen -- a ragged batch of images: the tokens of num_seqs
+ * images packed along one axis, each attending only within its own image.
+ * Source: inferencelayer "src/vision_gpu.rs", the vision tower's `forward`
+ * (attention over an image is one ragged segment given by its start
+ * offsets; several images are several segments).
+ *   q, k, v   device pointers, [total, H, D] of `dtype` (token-major, D
+ *             contiguous), total = cu_seqlens[num_seqs]; 16-byte aligned.
+ *   out       device pointer, [total, H, D], not overlapping q, k or v.
+ *             Every element of every token is written.
+ *   cu_seqlens  HOST pointer to num_seqs + 1 int32 offsets, cu_seqlens[0] = 0,
+ *             nondecreasing: segment s is tokens cu_seqlens[s] ..
+ *             cu_seqlens[s+1] - 1 (empty segments are allowed).  Read before
+ *             the call returns; not retained.
+ *   num_seqs  1 .. VITATTN_MAX_SEQS.
+ *   H, D, scale, dtype, stream: as for vitattn_forward.
+ * For token i of segment s and head h:
+ *     out[i,h,:] = softmax_j(scale * q[i,h,:] . k[j,h,:]) v[j,h,:], j in segment s.
+ * total = 0 enqueues nothing and returns VITATTN_OK.  Returns
+ * VITATTN_ERR_SEQLENS for malformed offsets, VITATTN_ERR_DIM for num_seqs out
+ * of range; other errors as for vitattn_forward.  Launches one kernel.
+ * A segment's key blocks may overlap the next segment's tokens in memory;
+ * those keys get probability 0, so values there must be finite (a NaN or inf
+ * in a neighbouring token's v can reach this segment's output as NaN).
+ */
+VITATTN_API int vitattn_forward_varlen(const void* q, const void* k, const void* v, void* out,
+                                       const int32_t* cu_seqlens, int64_t num_seqs, int64_t H, int64_t D,
+                                       float scale, int dtype, vitattn_stream_t stream);
+
+/* vitattn_forward_varlen, then a stream synchronisation and a read of the
+ * kernel's status words, as vitattn_forward_checked. */
+VITATTN_API int vitattn_forward_varlen_checked(const void* q, const void* k, const void* v, void* out,
+                                               const int32_t* cu_seqlens, int64_t num_seqs, int64_t H,
+                                               int64_t D, float scale, int dtype, vitattn_stream_t stream);
+
+/* The argument checks of vitattn_forward_varlen alone (no CUDA call). */
+VITATTN_API int vitattn_check_args_varlen(const void* q, const void* k, const void* v, const void* out,
+                                          const int32_t* cu_seqlens, int64_t num_seqs, int64_t H, int64_t D,
+                                          float scale, int dtype);
 
 /*
  * vitattn_forward_host -- the same operation from HOST buffers: enqueues the

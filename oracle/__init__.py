@@ -137,6 +137,26 @@ def attention_varlen(q, k, v, cu_seqlens, scale: float, dtype: int, mode: int = 
     return out
 
 
+def attention_varlen_rows(q, k, v, cu_seqlens, scale: float, dtype: int, rows,
+                          mode: int = MODE_TWO_PASS) -> np.ndarray:
+    """Selected output rows of :func:`attention_varlen`: ``rows`` holds flat
+    token-head indices ``i*H + h`` into ``[total, H]``; returns
+    ``[len(rows), D]`` float64 in the order given.  Each row is computed
+    over its own segment's keys only."""
+    cu = np.asarray([int(x) for x in cu_seqlens], dtype=np.int64)
+    H = q.shape[1]
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    tok = rows // H
+    seg = np.searchsorted(cu, tok, side="right") - 1
+    out = np.empty((rows.size, q.shape[2]), np.float64)
+    for s in np.unique(seg):
+        a, b = int(cu[s]), int(cu[s + 1])
+        sel = np.nonzero(seg == s)[0]
+        local = rows[sel] - a * H
+        out[sel] = attention_rows(q[None, a:b], k[None, a:b], v[None, a:b], scale, dtype, local, mode)
+    return out
+
+
 def widen(bits: np.ndarray, dtype: int) -> np.ndarray:
     """bf16 / f16 bit patterns to float64, exactly."""
     bits = np.ascontiguousarray(bits, dtype=np.uint16)

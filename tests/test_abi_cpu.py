@@ -100,3 +100,37 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(vitattn, "LIB_PATH", "/nonexistent/libvitattn.so")
     with pytest.raises(ImportError):
         vitattn.lib()
+
+
+# ---------------------------------------------------------------- ragged batches
+
+def check_var(cu=(0, 40, 64), **kw):
+    a = dict(q=Q, k=K, v=V, out=O, H=2, D=64, scale=0.125, dtype=vitattn.BF16)
+    a.update(kw)
+    return vitattn.check_args_varlen(a["q"], a["k"], a["v"], a["out"], list(cu), a["H"], a["D"], a["scale"],
+                                     a["dtype"])
+
+
+def test_varlen_valid_arguments_pass():
+    assert check_var() == 0
+    assert check_var(cu=(0, 0, 64)) == 0            # empty segments are allowed
+    assert check_var(cu=(0, 64)) == 0
+    assert check_var(cu=[0] + [1] * 255 + [2], D=16) == 0  # 256 segments
+    assert check_var(D=128, dtype=vitattn.F16) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(out=0), -1),
+    (dict(cu=(1, 40, 64)), -12), (dict(cu=(0, 40, 30)), -12), (dict(cu=(0, -1, 5)), -12),
+    (dict(cu=[0] * 258), -2), (dict(H=0), -2), (dict(cu=(0, 2**31 - 1)), -2),
+    (dict(D=60), -3), (dict(dtype=3), -4), (dict(q=Q + 4), -5),
+    (dict(out=K + 32), -6), (dict(scale=float("nan")), -9),
+])
+def test_varlen_argument_errors(kw, code):
+    assert check_var(**kw) == code
+    assert vitattn.strerror(code) not in ("ok", "unknown status")
+
+
+def test_varlen_with_no_tokens_is_a_no_op_without_cuda():
+    assert vitattn.forward_varlen_ptr(Q, K, V, O, [0, 0, 0], 2, 64, 0.125, vitattn.BF16) == 0
+    assert vitattn.forward_varlen_ptr(Q, K, V, O, [0, 5, 3], 2, 64, 0.125, vitattn.BF16) == -12

@@ -359,3 +359,11 @@ def test_varlen_oracle_rejects_bad_offsets():
     for cu in ([1, 4], [0, 3, 2, 4], [0, 3]):
         with pytest.raises(ValueError):
             oracle.attention_varlen(q, q, q, cu, 1.0, oracle.BF16)
+
+
+def test_varlen_rows_match_the_full_varlen_output():
+    cu = [0, 3, 3, 11, 16]
+    q, k, v = (synth.round_to_bits(rnd((16, 3, 8), 97 + i).astype(np.float32), synth.F16) for i in range(3))
+    full = oracle.attention_varlen(q, k, v, cu, 0.3, oracle.F16).reshape(16 * 3, 8)
+    rows = np.array([47, 0, 9, 10, 30, 8, 33])
+    assert np.array_equal(oracle.attention_varlen_rows(q, k, v, cu, 0.3, oracle.F16, rows), full[rows])

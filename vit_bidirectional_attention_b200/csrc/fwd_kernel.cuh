@@ -175,14 +175,33 @@ __host__ __device__ constexpr int smem_bytes(int dp, bool loop) {
     return (q_buffers(dp, loop) * kTilesPerCta + kStages) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
 }
 
+// Ragged batches (several images' tokens packed along one axis, start
+// offsets cu_seqlens): segment s is tokens start[s] .. start[s] + len[s] - 1,
+// and its work items (head, group of query tiles) are item0[s] ..
+// item0[s+1] - 1, qgroups[s] query groups per head.  The dense layout needs
+// none of it (an empty table).
+constexpr int kMaxSegs = 256;
+template <bool kVarlen>
+struct SegTable {
+    int n;
+};
+template <>
+struct SegTable<true> {
+    int n;                    // segments
+    int start[kMaxSegs];      // first token of segment s
+    int len[kMaxSegs];        // its token count
+    int qgroups[kMaxSegs];    // ceil(len / (128 * tiles_per_cta))
+    int item0[kMaxSegs + 1];  // first work item of segment s; item0[n] = all items
+};
+
 struct alignas(64) FwdParams {
     CUtensorMap maps[3][3];  // [q, k, v][width class 64 / 32 / 16]
     void* out;
     int B, N, H, D;
     int tiles_per_cta;  // query tiles a work item owns: 2, or 1 when 2 would leave SMs idle
-    int n_qgroups;      // ceil(N / (128 * tiles_per_cta)): work items per (b, h)
-    int n_items;        // B * H * n_qgroups; a CTA takes items blockIdx.x + k * gridDim.x
-    int n_kblocks;      // ceil(N / 128)
+    int n_qgroups;      // ceil(N / (128 * tiles_per_cta)): work items per (b, h) (dense layout)
+    int n_items;        // all work items; a CTA takes items blockIdx.x + k * gridDim.x
+    int n_kblocks;      // ceil(N / 128) (dense layout; a ragged batch takes it per segment)
     float scale_log2;
     int flags;
     unsigned long long timeout_ns;
@@ -474,11 +493,16 @@ __device__ __forceinline__ void store_row(uint32_t tO, float inv_l, uint8_t* oro
 
 // kLoop: the CTA loops over work items (grid smaller than the item count);
 // without it every CTA owns exactly one item and the item loops fold away.
-template <int DP, bool kBF16, bool kLoop>
-__global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
+// kVarlen: a ragged batch (tokens of several images packed along the N axis
+// of a B = 1 tensor, described by `seg`); each work item attends within its
+// own segment.  Ragged batches run one item per CTA.
+template <int DP, bool kBF16, bool kLoop, bool kVarlen>
+__global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p,
+                                                          const __grid_constant__ SegTable<kVarlen> seg) {
     constexpr int TILE = tile_bytes(DP);
     constexpr int NCH = chunk_count(DP);
     static_assert(DP % 16 == 0 && DP >= 16 && DP <= 128, "head dim padding");
+    static_assert(!(kLoop && kVarlen), "ragged batches run one work item per CTA");
 
     constexpr int NQ = q_buffers(DP, kLoop);
     extern __shared__ uint8_t smem_raw[];
@@ -496,27 +520,50 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work items: (b, h, group of query tiles), numbered so that the items of
-    // one (b, h) are adjacent and the CTAs running at once share K/V in L2.
-    // This CTA takes items blockIdx.x, blockIdx.x + gridDim.x, ...; the host
-    // launches fewer CTAs than items only when every item has the same number
-    // of query tiles, so T below holds for all of this CTA's items.
+    // Work items: (b, h, group of query tiles) -- for a ragged batch (segment,
+    // h, group) -- numbered so that the items of one (b, h) are adjacent and
+    // the CTAs running at once share K/V in L2.  An item attends over the n
+    // tokens starting at token tok0 of batch b.  This CTA takes items
+    // blockIdx.x, blockIdx.x + gridDim.x, ...; the host launches fewer CTAs
+    // than items only when every item has the same number of query tiles and
+    // key blocks, so T and nkb below hold for all of this CTA's items.
     struct Item {
-        int b, h, q0, nt;
+        int b, h, q0, nt, tok0, n;
     };
     auto item_of = [&](int i) -> Item {
         Item it;
-        const int qg = i % p.n_qgroups;
-        const int bh = i / p.n_qgroups;
-        it.h = bh % p.H;
-        it.b = bh / p.H;
+        int qg;
+        if constexpr (kVarlen) {
+            // the segment whose items contain i: the last s with item0[s] <= i
+            // (an empty segment has no items, so it is never the answer)
+            int lo = 0, hi = seg.n;
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (seg.item0[mid] <= i) lo = mid;
+                else hi = mid;
+            }
+            const int local = i - seg.item0[lo];
+            it.h = local / seg.qgroups[lo];
+            qg = local - it.h * seg.qgroups[lo];
+            it.b = 0;
+            it.tok0 = seg.start[lo];
+            it.n = seg.len[lo];
+        } else {
+            qg = i % p.n_qgroups;
+            const int bh = i / p.n_qgroups;
+            it.h = bh % p.H;
+            it.b = bh / p.H;
+            it.tok0 = 0;
+            it.n = p.N;
+        }
         it.q0 = qg * (p.tiles_per_cta * kTileRows);
-        it.nt = (p.tiles_per_cta == 2 && it.q0 + kTileRows < p.N) ? 2 : 1;
+        it.nt = (p.tiles_per_cta == 2 && it.q0 + kTileRows < it.n) ? 2 : 1;
         return it;
     };
     const int n_my = kLoop ? (p.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 1;
-    const int T = item_of(blockIdx.x).nt;
-    const int nkb = p.n_kblocks;
+    const Item first = item_of(blockIdx.x);
+    const int T = first.nt;
+    const int nkb = kLoop ? p.n_kblocks : (first.n + kBlockKeys - 1) / kBlockKeys;
     const uint64_t tmo = p.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -581,7 +628,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                     for (int c = 0; c < NCH; ++c)
                         ptx::tma_load_4d(sQ + (qb * kTilesPerCta + t) * TILE + 256 * chunk_col(DP, c),
                                          &p.maps[0][width_class(chunk_width(DP, c))], chunk_col(DP, c),
-                                         it.h, it.q0 + t * kTileRows, it.b, bar(kBarQFull + 2 * qb + t));
+                                         it.h, it.tok0 + it.q0 + t * kTileRows, it.b,
+                                         bar(kBarQFull + 2 * qb + t));
                     q_last[t] = k;
                 }
 
@@ -599,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                         for (int c = 0; c < NCH; ++c)
                             ptx::tma_load_4d(sKV + slot * TILE + 256 * chunk_col(DP, c),
                                              &p.maps[1 + kv][width_class(chunk_width(DP, c))],
-                                             chunk_col(DP, c), it.h, j * kBlockKeys, it.b,
+                                             chunk_col(DP, c), it.h, it.tok0 + j * kBlockKeys, it.b,
                                              bar(kBarKvFull + slot));
                     }
                 }
@@ -839,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
                         for (int i = 0; i < 32; ++i) s[32 * q + i] = __uint_as_float(r[q][i]);
                 }
-                const int valid = min(kBlockKeys, p.N - j * kBlockKeys);
+                const int valid = min(kBlockKeys, it.n - j * kBlockKeys);
                 const bool partial = valid < kBlockKeys;
                 const float ext = partial ? (neg ? row_extreme<true, true>(s, valid)
                                                  : row_extreme<true, false>(s, valid))
@@ -876,9 +924,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             if (ok) ok = wait_warp(bar(kBarOFull + t), (uint32_t)k & 1u, abort_flag, tmo, 8);
             if (ok) {
                 ptx::tc_fence_after();
-                uint8_t* orow = reinterpret_cast<uint8_t*>(p.out) +
-                                ((((size_t)it.b * p.N + (size_t)min(row, p.N - 1)) * p.H + it.h) * p.D) * 2;
-                store_row<DP, kBF16>(tO, 1.f / l, orow, row < p.N, p.D);
+                uint8_t* orow =
+                    reinterpret_cast<uint8_t*>(p.out) +
+                    ((((size_t)it.b * p.N + (size_t)it.tok0 + (size_t)min(row, it.n - 1)) * p.H + it.h) * p.D) * 2;
+                store_row<DP, kBF16>(tO, 1.f / l, orow, row < it.n, p.D);
                 // O_t has been read (store_row waits for each load): the next
                 // item's first P.V may overwrite it
                 if (kLoop) {

@@ -17,6 +17,9 @@
 namespace {
 
 using vitattn::FwdParams;
+using SegDense = vitattn::SegTable<false>;
+using SegVar = vitattn::SegTable<true>;
+static_assert(vitattn::kMaxSegs == VITATTN_MAX_SEQS, "segment table size");
 
 constexpr int kVersion = 10000;  // 1.0.0
 constexpr int kMaxDevices = 64;
@@ -55,6 +58,37 @@ int check_args(const void* q, const void* k, const void* v, const void* out, int
     if (mis) return VITATTN_ERR_ALIGN;
     const uint64_t bytes = batch_stride * (uint64_t)B;
     if (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes))
+        return VITATTN_ERR_ALIAS;
+    return VITATTN_OK;
+}
+
+// Ragged batch: q, k, v, out are [total, H, D] with total = cu_seqlens[num_seqs];
+// cu_seqlens (host) starts at 0 and never decreases.
+int check_args_varlen(const void* q, const void* k, const void* v, const void* out,
+                      const int32_t* cu_seqlens, int64_t num_seqs, int64_t H, int64_t D, float scale,
+                      int dtype) {
+    if (!q || !k || !v || !out || !cu_seqlens) return VITATTN_ERR_NULL;
+    if (num_seqs < 1 || num_seqs > vitattn::kMaxSegs || H < 1 || D < 1) return VITATTN_ERR_DIM;
+    if (D < 16 || D > 128 || D % 8 != 0) return VITATTN_ERR_HEADDIM;
+    if (dtype != VITATTN_BF16 && dtype != VITATTN_F16) return VITATTN_ERR_DTYPE;
+    if (!std::isfinite(scale)) return VITATTN_ERR_SCALE;
+    if (cu_seqlens[0] != 0) return VITATTN_ERR_SEQLENS;
+    for (int64_t s = 0; s < num_seqs; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return VITATTN_ERR_SEQLENS;
+    const int64_t total = cu_seqlens[num_seqs];
+    // TMA token coordinates and per-item token offsets are int32
+    if (total > (int64_t)INT32_MAX - 512 || H > (int64_t)INT32_MAX) return VITATTN_ERR_DIM;
+    const uint64_t token_bytes = (uint64_t)H * (uint64_t)D * 2u;
+    if (token_bytes >= (1ull << 40) || (uint64_t)total > (1ull << 62) / token_bytes) return VITATTN_ERR_DIM;
+    uint64_t work = 0;
+    for (int64_t s = 0; s < num_seqs; ++s)
+        work += (uint64_t)H * (uint64_t)((cu_seqlens[s + 1] - cu_seqlens[s] + 127) / 128);
+    if (work > (uint64_t)INT32_MAX) return VITATTN_ERR_DIM;
+    const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                           reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out)) & 15u;
+    if (mis) return VITATTN_ERR_ALIGN;
+    const uint64_t bytes = token_bytes * (uint64_t)total;
+    if (bytes > 0 && (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)))
         return VITATTN_ERR_ALIAS;
     return VITATTN_OK;
 }
@@ -99,25 +133,35 @@ bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t N
 
 // ---------------------------------------------------------------- dispatch
 
-using KernelFn = void (*)(FwdParams);
+// Kernel modes: one work item per CTA, CTAs looping over items, ragged batch.
+enum Mode { kModeItem = 0, kModeLoop = 1, kModeVarlen = 2, kNumModes = 3 };
 
 template <int DP>
-KernelFn kernel_of(bool bf, bool loop) {
-    if (bf) return loop ? vitattn::fwd_kernel<DP, true, true> : vitattn::fwd_kernel<DP, true, false>;
-    return loop ? vitattn::fwd_kernel<DP, false, true> : vitattn::fwd_kernel<DP, false, false>;
+const void* kernel_of(bool bf, Mode mode) {
+    switch (mode) {
+        case kModeLoop:
+            return bf ? reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, true, true, false>)
+                      : reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, false, true, false>);
+        case kModeVarlen:
+            return bf ? reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, true, false, true>)
+                      : reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, false, false, true>);
+        default:
+            return bf ? reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, true, false, false>)
+                      : reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, false, false, false>);
+    }
 }
 
-KernelFn pick_kernel(int dp, int dtype, bool loop) {
+const void* pick_kernel(int dp, int dtype, Mode mode) {
     const bool bf = dtype == VITATTN_BF16;
     switch (dp) {
-        case 16: return kernel_of<16>(bf, loop);
-        case 32: return kernel_of<32>(bf, loop);
-        case 48: return kernel_of<48>(bf, loop);
-        case 64: return kernel_of<64>(bf, loop);
-        case 80: return kernel_of<80>(bf, loop);
-        case 96: return kernel_of<96>(bf, loop);
-        case 112: return kernel_of<112>(bf, loop);
-        case 128: return kernel_of<128>(bf, loop);
+        case 16: return kernel_of<16>(bf, mode);
+        case 32: return kernel_of<32>(bf, mode);
+        case 48: return kernel_of<48>(bf, mode);
+        case 64: return kernel_of<64>(bf, mode);
+        case 80: return kernel_of<80>(bf, mode);
+        case 96: return kernel_of<96>(bf, mode);
+        case 112: return kernel_of<112>(bf, mode);
+        case 128: return kernel_of<128>(bf, mode);
         default: return nullptr;
     }
 }
@@ -128,7 +172,7 @@ struct DeviceState {
     bool checked = false;
     bool is_sm100 = false;
     int num_sms = 0;
-    bool smem_set[9][2][2] = {};
+    bool smem_set[9][2][kNumModes] = {};
 };
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -158,19 +202,57 @@ int device_info(int* num_sms) {
 }
 
 // The dynamic shared-memory limit of one kernel instantiation, raised once per device.
-int ensure_smem(int dp, int dtype, bool loop, KernelFn fn) {
+int ensure_smem(int dp, int dtype, Mode mode, const void* fn) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     std::lock_guard<std::mutex> lock(g_mu);
-    bool& done = g_dev[dev].smem_set[dp / 16][dtype][loop ? 1 : 0];
+    bool& done = g_dev[dev].smem_set[dp / 16][dtype][mode];
     if (!done) {
-        e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fn),
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 vitattn::smem_bytes(dp, loop));
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 vitattn::smem_bytes(dp, mode == kModeLoop));
         if (e != cudaSuccess) return cuda_fail(e);
         done = true;
     }
+    return VITATTN_OK;
+}
+
+// Tensor maps of q, k, v for every column-chunk width, and the shape fields.
+int fill_common(FwdParams* prm, const void* q, const void* k, const void* v, void* out, int64_t B,
+                int64_t N, int64_t H, int64_t D, float scale, int dtype, int flags) {
+    std::memset(prm, 0, sizeof *prm);
+    const int dp = (int)((D + 15) / 16 * 16);
+    const void* src[3] = {q, k, v};
+    const int nch = vitattn::chunk_count(dp);
+    for (int c = 0; c < nch; ++c) {
+        const int w = vitattn::chunk_width(dp, c);
+        for (int m = 0; m < 3; ++m) {
+            CUtensorMap* map = &prm->maps[m][vitattn::width_class(w)];
+            if (!encode_map(map, src[m], dtype, B, N, H, D, w)) return cuda_fail(cudaErrorInvalidValue);
+        }
+    }
+    prm->out = out;
+    prm->B = (int)B;
+    prm->N = (int)N;
+    prm->H = (int)H;
+    prm->D = (int)D;
+    prm->scale_log2 = (float)((double)scale * 1.4426950408889634);
+    prm->flags = flags;
+    prm->timeout_ns = kWaitTimeoutNs;
+    return VITATTN_OK;
+}
+
+template <class Seg>
+int run_kernel(int dp, int dtype, Mode mode, unsigned grid, FwdParams* prm, Seg* seg,
+               cudaStream_t stream) {
+    const void* fn = pick_kernel(dp, dtype, mode);
+    if (!fn) return VITATTN_ERR_HEADDIM;
+    int rc = ensure_smem(dp, dtype, mode, fn);
+    if (rc) return rc;
+    void* args[2] = {prm, seg};
+    cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(vitattn::kThreads), args,
+                                     (size_t)vitattn::smem_bytes(dp, mode == kModeLoop), stream);
+    if (e != cudaSuccess) return cuda_fail(e);
     return VITATTN_OK;
 }
 
@@ -184,21 +266,8 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     if (rc) return rc;
 
     FwdParams prm;
-    std::memset(&prm, 0, sizeof prm);
-    const void* src[3] = {q, k, v};
-    const int nch = vitattn::chunk_count(dp);
-    for (int c = 0; c < nch; ++c) {
-        const int w = vitattn::chunk_width(dp, c);
-        for (int m = 0; m < 3; ++m) {
-            CUtensorMap* map = &prm.maps[m][vitattn::width_class(w)];
-            if (!encode_map(map, src[m], dtype, B, N, H, D, w)) return cuda_fail(cudaErrorInvalidValue);
-        }
-    }
-    prm.out = out;
-    prm.B = (int)B;
-    prm.N = (int)N;
-    prm.H = (int)H;
-    prm.D = (int)D;
+    rc = fill_common(&prm, q, k, v, out, B, N, H, D, scale, dtype, flags);
+    if (rc) return rc;
     // Two query tiles per CTA share each K/V block (fewer K/V reads, two
     // softmax warpgroups in flight); one per CTA when two would leave SMs idle.
     const uint64_t pairs = (uint64_t)B * (uint64_t)H * (uint64_t)((N + 255) / 256);
@@ -208,9 +277,6 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     prm.n_qgroups = (int)((N + 128 * prm.tiles_per_cta - 1) / (128 * prm.tiles_per_cta));
     prm.n_items = (int)((uint64_t)B * (uint64_t)H * (uint64_t)prm.n_qgroups);
     prm.n_kblocks = (int)((N + 127) / 128);
-    prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    prm.flags = flags;
-    prm.timeout_ns = kWaitTimeoutNs;
 
     // Persistent grid (one CTA per SM, each looping over work items) when there
     // are more items than SMs, the items are short enough (at most 32 key
@@ -223,22 +289,52 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     if (uniform && (flags & vitattn::kFlagTinyGrid) && grid > 3u) grid = 3u;
     const bool loop = grid < (unsigned)prm.n_items;
 
-    KernelFn fn = pick_kernel(dp, dtype, loop);
-    if (!fn) return VITATTN_ERR_HEADDIM;
-    rc = ensure_smem(dp, dtype, loop, fn);
-    if (rc) return rc;
-    void* args[1] = {&prm};
-    cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(fn), dim3(grid),
-                                     dim3(vitattn::kThreads), args,
-                                     (size_t)vitattn::smem_bytes(dp, loop), stream);
-    if (e != cudaSuccess) return cuda_fail(e);
-    return VITATTN_OK;
+    SegDense seg{0};
+    return run_kernel(dp, dtype, loop ? kModeLoop : kModeItem, grid, &prm, &seg, stream);
 }
 
-int forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
-                    int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags) {
-    int rc = check_args(q, k, v, out, B, N, H, D, scale, dtype);
+// Ragged batch: one CTA per work item (segment, head, group of query tiles).
+int launch_varlen(const void* q, const void* k, const void* v, void* out, const int32_t* cu,
+                  int64_t num_seqs, int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream,
+                  int flags) {
+    int rc = check_args_varlen(q, k, v, out, cu, num_seqs, H, D, scale, dtype);
     if (rc) return rc;
+    const int64_t total = cu[num_seqs];
+    if (total == 0) return VITATTN_OK;  // no tokens: nothing to compute or write
+    const int dp = (int)((D + 15) / 16 * 16);
+    int num_sms = 0;
+    rc = device_info(&num_sms);
+    if (rc) return rc;
+
+    FwdParams prm;
+    rc = fill_common(&prm, q, k, v, out, 1, total, H, D, scale, dtype, flags);
+    if (rc) return rc;
+    static thread_local SegVar seg;  // ~4 KB: kept off the stack
+    std::memset(&seg, 0, sizeof seg);
+    seg.n = (int)num_seqs;
+    // two query tiles per item unless that leaves SMs idle (as for the dense layout)
+    uint64_t pairs = 0;
+    for (int64_t s = 0; s < num_seqs; ++s) pairs += (uint64_t)H * (uint64_t)((cu[s + 1] - cu[s] + 255) / 256);
+    int tiles = pairs < (uint64_t)num_sms ? 1 : 2;
+    if (flags & vitattn::kFlagForceTwoTiles) tiles = 2;
+    if (flags & vitattn::kFlagForceOneTile) tiles = 1;
+    int items = 0;
+    for (int s = 0; s < (int)num_seqs; ++s) {
+        seg.start[s] = cu[s];
+        seg.len[s] = cu[s + 1] - cu[s];
+        seg.qgroups[s] = (seg.len[s] + 128 * tiles - 1) / (128 * tiles);
+        seg.item0[s] = items;
+        items += (int)H * seg.qgroups[s];
+    }
+    seg.item0[num_seqs] = items;
+    prm.tiles_per_cta = tiles;
+    prm.n_items = items;
+    return run_kernel(dp, dtype, kModeVarlen, (unsigned)items, &prm, &seg, stream);
+}
+
+// Launch (through `go`), synchronise, and read the kernel's status words.
+template <class Go>
+int checked_run(cudaStream_t stream, Go go) {
     const unsigned zero = 0;
     cudaError_t e = cudaMemcpyToSymbolAsync(g_vitattn_status, &zero, sizeof zero, 0,
                                             cudaMemcpyHostToDevice, stream);
@@ -246,7 +342,7 @@ int forward_checked(const void* q, const void* k, const void* v, void* out, int6
     e = cudaMemcpyToSymbolAsync(g_vitattn_range, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,
                                 stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    rc = launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags);
+    int rc = go();
     if (rc) return rc;
     e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return cuda_fail(e);
@@ -257,6 +353,23 @@ int forward_checked(const void* q, const void* k, const void* v, void* out, int6
     if (e != cudaSuccess) return cuda_fail(e);
     if (status) return VITATTN_ERR_TIMEOUT;
     return range ? VITATTN_ERR_RANGE : VITATTN_OK;
+}
+
+int forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
+                    int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags) {
+    int rc = check_args(q, k, v, out, B, N, H, D, scale, dtype);
+    if (rc) return rc;
+    return checked_run(stream, [&] { return launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags); });
+}
+
+int forward_varlen_checked(const void* q, const void* k, const void* v, void* out, const int32_t* cu,
+                           int64_t num_seqs, int64_t H, int64_t D, float scale, int dtype,
+                           cudaStream_t stream, int flags) {
+    int rc = check_args_varlen(q, k, v, out, cu, num_seqs, H, D, scale, dtype);
+    if (rc) return rc;
+    return checked_run(stream, [&] {
+        return launch_varlen(q, k, v, out, cu, num_seqs, H, D, scale, dtype, stream, flags);
+    });
 }
 
 }  // namespace
@@ -285,6 +398,36 @@ VITATTN_API int vitattn_test_forward_flags(const void* q, const void* k, const v
                                vitattn_stream_t stream, int flags) {
     return forward_checked(q, k, v, out, B, N, H, D, scale, dtype,
                            reinterpret_cast<cudaStream_t>(stream), flags);
+}
+
+int vitattn_forward_varlen(const void* q, const void* k, const void* v, void* out,
+                           const int32_t* cu_seqlens, int64_t num_seqs, int64_t H, int64_t D, float scale,
+                           int dtype, vitattn_stream_t stream) {
+    return launch_varlen(q, k, v, out, cu_seqlens, num_seqs, H, D, scale, dtype,
+                         reinterpret_cast<cudaStream_t>(stream), 0);
+}
+
+int vitattn_forward_varlen_checked(const void* q, const void* k, const void* v, void* out,
+                                   const int32_t* cu_seqlens, int64_t num_seqs, int64_t H, int64_t D,
+                                   float scale, int dtype, vitattn_stream_t stream) {
+    return forward_varlen_checked(q, k, v, out, cu_seqlens, num_seqs, H, D, scale, dtype,
+                                  reinterpret_cast<cudaStream_t>(stream), 0);
+}
+
+// Test hook, deliberately absent from the public header: the checked ragged
+// entry with the test flags of vitattn_test_forward_flags.
+VITATTN_API int vitattn_test_forward_varlen_flags(const void* q, const void* k, const void* v, void* out,
+                                                  const int32_t* cu_seqlens, int64_t num_seqs, int64_t H,
+                                                  int64_t D, float scale, int dtype, vitattn_stream_t stream,
+                                                  int flags) {
+    return forward_varlen_checked(q, k, v, out, cu_seqlens, num_seqs, H, D, scale, dtype,
+                                  reinterpret_cast<cudaStream_t>(stream), flags);
+}
+
+int vitattn_check_args_varlen(const void* q, const void* k, const void* v, const void* out,
+                              const int32_t* cu_seqlens, int64_t num_seqs, int64_t H, int64_t D,
+                              float scale, int dtype) {
+    return check_args_varlen(q, k, v, out, cu_seqlens, num_seqs, H, D, scale, dtype);
 }
 
 int vitattn_forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq,
@@ -326,6 +469,7 @@ const char* vitattn_strerror(int status) {
         case VITATTN_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
         case VITATTN_ERR_SCALE: return "scale must be finite";
         case VITATTN_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+        case VITATTN_ERR_SEQLENS: return "cu_seqlens must start at 0 and never decrease";
         case VITATTN_ERR_RANGE: return "a bf16 V value has magnitude >= 65536, outside the f16 P.V product's range";
         default: return "unknown status";
     }

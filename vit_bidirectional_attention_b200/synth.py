@@ -21,6 +21,16 @@ Workloads (token-major ``[B, N, H, D]`` as they leave a ViT's QKV linear):
   so that a logit q.k/sqrt(D) has variance 1 + (16a^2 + 8a^4)/D = 16 (std 4:
   a peaky softmax that keeps raising the running maximum); V iid N(0,1).
 
+Ragged batches (several images' tokens packed along one axis, ``[total, H, D]``
+with ``cu_seqlens`` start offsets, each image attending only within itself):
+
+- ``multi_image``  20 images of 1024, 576, 256, 912, 196, 4096, 729, 1600, 2304,
+  400, 784, 1369, 3136, 64, 2025, 900, 1156, 484, 2601 and 324 patches
+  (24 936 tokens: square patch grids from 8^2 to 64^2 and the 912-patch
+  page, the mixed resolutions a dynamic-resolution ViT sees; 243 MiB of
+  inputs and output, more than the 126 MiB L2), 16 heads, D = 80, bf16,
+  Q,K iid N(0, 1.5^2), V iid N(0,1) (the ``doc_page`` distribution).
+
 Every workload uses scale = 1/sqrt(D) and seed 20261202 + its index.
 """
 from __future__ import annotations
@@ -80,6 +90,79 @@ WORKLOADS = {
         Workload("high_res", 2, 16384, 16, 128, BF16, rank8_logit_std=4.0, index=4),
     )
 }
+
+
+@dataclasses.dataclass(frozen=True)
+class RaggedWorkload:
+    name: str
+    seqlens: tuple
+    H: int
+    D: int
+    dtype: int
+    qk_std: float = 1.0
+    index: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def seed(self) -> int:
+        return SEED_BASE + self.index
+
+    @property
+    def cu_seqlens(self) -> list:
+        cu = [0]
+        for n in self.seqlens:
+            cu.append(cu[-1] + n)
+        return cu
+
+    @property
+    def total(self) -> int:
+        return sum(self.seqlens)
+
+    @property
+    def flops(self) -> float:
+        """4*H*D*sum(n_s^2): each image's QK^T and PV, two flops per MAC."""
+        return 4.0 * self.H * self.D * sum(n * n for n in self.seqlens)
+
+    @property
+    def io_bytes(self) -> int:
+        return 4 * self.total * self.H * self.D * 2
+
+    @property
+    def numel(self) -> int:
+        return self.total * self.H * self.D
+
+
+RAGGED = {
+    w.name: w
+    for w in (
+        RaggedWorkload("multi_image", (1024, 576, 256, 912, 196, 4096, 729, 1600, 2304, 400,
+                                       784, 1369, 3136, 64, 2025, 900, 1156, 484, 2601, 324), 16, 80, BF16,
+                       qk_std=1.5, index=5),
+    )
+}
+
+
+def make_qkv_ragged(w: RaggedWorkload, seed: int | None = None):
+    """(q, k, v) uint16 bit arrays of shape [total, H, D] for ragged workload ``w``."""
+    rng = np.random.Generator(np.random.PCG64(w.seed if seed is None else seed))
+    shape = (w.total, w.H, w.D)
+    out = []
+    for std in (w.qk_std, w.qk_std, 1.0):
+        x = rng.standard_normal(size=shape, dtype=np.float32)
+        if std != 1.0:
+            x *= np.float32(std)
+        out.append(round_to_bits(x, w.dtype))
+    return tuple(out)
+
+
+def random_ragged(seqlens, H: int, D: int, dtype: int, seed: int, std: float = 1.0):
+    """iid N(0, std^2) ragged inputs ``[total, H, D]`` and their cu_seqlens."""
+    w = RaggedWorkload("sweep", tuple(int(n) for n in seqlens), H, D, dtype, qk_std=std)
+    q, k, v = make_qkv_ragged(w, seed=seed)
+    return q, k, v, w.cu_seqlens
 
 
 def round_to_bits(x: np.ndarray, dtype: int) -> np.ndarray:

@@ -27,6 +27,7 @@ STATUS_NAMES = {
     -9: "VITATTN_ERR_SCALE",
     -10: "VITATTN_ERR_DEVICE",
     -11: "VITATTN_ERR_RANGE",
+    -12: "VITATTN_ERR_SEQLENS",
 }
 
 _lib = None
@@ -56,11 +57,18 @@ def lib() -> ctypes.CDLL:
         L.vitattn_test_forward_flags.argtypes = fwd + [i32]
         L.vitattn_forward_host.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, f32, i32, p]
         L.vitattn_check_args.argtypes = [p, p, p, p, i64, i64, i64, i64, f32, i32]
+        var = [p, p, p, p, p, i64, i64, i64, f32, i32, p]
+        L.vitattn_forward_varlen.argtypes = var
+        L.vitattn_forward_varlen_checked.argtypes = var
+        L.vitattn_test_forward_varlen_flags.argtypes = var + [i32]
+        L.vitattn_check_args_varlen.argtypes = var[:-1]
         L.vitattn_strerror.argtypes = [i32]
         L.vitattn_strerror.restype = ctypes.c_char_p
         for f in (L.vitattn_forward, L.vitattn_forward_checked, L.vitattn_test_forward_flags,
                   L.vitattn_forward_host, L.vitattn_check_args, L.vitattn_last_cuda_error,
-                  L.vitattn_version, L.vitattn_launches_per_call):
+                  L.vitattn_version, L.vitattn_launches_per_call, L.vitattn_forward_varlen,
+                  L.vitattn_forward_varlen_checked, L.vitattn_test_forward_varlen_flags,
+                  L.vitattn_check_args_varlen):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -144,4 +152,77 @@ def forward(q, k, v, out=None, scale=None, stream=None, checked=False):
                          scale, dtype, handle, checked=checked)
     if rc != 0:
         raise VitAttnError(rc, "vitattn_forward")
+    return out
+
+
+MAX_SEQS = 256
+
+
+def _cu_array(cu_seqlens):
+    """cu_seqlens as a C int32 array (host memory) and the segment count."""
+    vals = [int(x) for x in cu_seqlens]
+    if len(vals) < 2:
+        raise ValueError("cu_seqlens needs at least two offsets")
+    arr = (ctypes.c_int32 * len(vals))(*vals)
+    return arr, len(vals) - 1
+
+
+def check_args_varlen(q, k, v, out, cu_seqlens, H, D, scale, dtype) -> int:
+    """Status the library's ragged-batch argument checks give; no CUDA call."""
+    arr, n = _cu_array(cu_seqlens)
+    return int(lib().vitattn_check_args_varlen(q, k, v, out, ctypes.cast(arr, ctypes.c_void_p), n, H, D,
+                                               float(scale), dtype))
+
+
+def forward_varlen_ptr(q, k, v, out, cu_seqlens, H, D, scale, dtype, stream=0, checked=False, flags=0) -> int:
+    """Raw ragged-batch call on device pointers (ints) and host offsets; returns the status."""
+    L = lib()
+    arr, n = _cu_array(cu_seqlens)
+    args = (q, k, v, out, ctypes.cast(arr, ctypes.c_void_p), n, H, D, float(scale), dtype, stream)
+    if flags:
+        return int(L.vitattn_test_forward_varlen_flags(*args, int(flags)))
+    if checked:
+        return int(L.vitattn_forward_varlen_checked(*args))
+    return int(L.vitattn_forward_varlen(*args))
+
+
+def forward_varlen(q, k, v, cu_seqlens, out=None, scale=None, stream=None, checked=False):
+    """Attention within each image of a ragged batch on CUDA tensors.
+
+    q, k, v: contiguous ``[total, H, D]`` bf16 / f16 CUDA tensors holding the
+    tokens of several images back to back; ``cu_seqlens`` (a host sequence of
+    ints, first 0, nondecreasing, last ``total``) gives where each image
+    starts.  Every token attends only to the keys of its own image.
+    ``scale`` defaults to 1/sqrt(D).  Returns ``out``.
+    """
+    import torch
+
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [total, H, D] shape")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous [total, H, D]")
+    dtype = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    if hasattr(cu_seqlens, "tolist"):
+        cu_seqlens = cu_seqlens.tolist()
+    total, H, D = q.shape
+    if int(cu_seqlens[-1]) != total:
+        raise ValueError("cu_seqlens must end at the token count")
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor like q")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    with torch.cuda.device(q.device):
+        rc = forward_varlen_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), cu_seqlens, H, D,
+                                scale, dtype, handle, checked=checked)
+    if rc != 0:
+        raise VitAttnError(rc, "vitattn_forward_varlen")
     return out
