@@ -157,6 +157,37 @@ def attention_varlen_rows(q, k, v, cu_seqlens, scale: float, dtype: int, rows,
     return out
 
 
+def qkv_rope(qkv, cos, sin, dtype: int):
+    """Split a packed QKV projection and apply the rotary embedding to q and k
+    (inferencelayer ``src/vision_gpu.rs``, ``VIS_QKV_ROPE`` and its doc: the
+    projection output is ``[rows, 3*hid]`` = q | k | v per token; the rope
+    tables ``cos``/``sin`` are ``[rows, head_dim]`` and arrive precomputed
+    (the 2-D row/column walk lives in whoever built them); element ``d`` of a
+    head pairs with ``d +- head_dim/2`` through ``rotate_half``, negated on
+    the low half; v is not rotated).
+
+    ``qkv``: ``[T, 3, H, D]`` bit patterns of ``dtype`` (or float64 with
+    ``dtype`` F64); ``cos``, ``sin``: ``[T, D]`` float32 (or float64).
+    Returns (q, k, v) as float64 ``[T, H, D]``, unrounded::
+
+        x'[d] = x[d] * cos[d] + rotate_half(x)[d] * sin[d]
+        rotate_half(x)[d] = -x[d + D/2]  (d < D/2),   x[d - D/2]  (d >= D/2)
+    """
+    T, three, H, D = qkv.shape
+    if three != 3 or D % 2:
+        raise ValueError("qkv must be [T, 3, H, D] with D even")
+    x = qkv.astype(np.float64) if dtype == F64 else widen(np.ascontiguousarray(qkv), dtype)
+    c = np.asarray(cos, np.float64)[:, None, :]
+    s = np.asarray(sin, np.float64)[:, None, :]
+    half = D // 2
+
+    def rope(t):
+        rot = np.concatenate([-t[..., half:], t[..., :half]], axis=-1)
+        return t * c + rot * s
+
+    return rope(x[:, 0]), rope(x[:, 1]), x[:, 2].copy()
+
+
 def widen(bits: np.ndarray, dtype: int) -> np.ndarray:
     """bf16 / f16 bit patterns to float64, exactly."""
     bits = np.ascontiguousarray(bits, dtype=np.uint16)

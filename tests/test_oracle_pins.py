@@ -367,3 +367,60 @@ def test_varlen_rows_match_the_full_varlen_output():
     full = oracle.attention_varlen(q, k, v, cu, 0.3, oracle.F16).reshape(16 * 3, 8)
     rows = np.array([47, 0, 9, 10, 30, 8, 33])
     assert np.array_equal(oracle.attention_varlen_rows(q, k, v, cu, 0.3, oracle.F16, rows), full[rows])
+
+
+# ---------------------------------------------------------------- QKV split + rotary embedding prologue
+
+def _rope_case(T, H, D, seed, dtype=synth.BF16):
+    qkv = synth.round_to_bits(rnd((T, 3, H, D), seed).astype(np.float32), dtype)
+    theta = rnd((T, D // 2), seed + 1)
+    ang = np.concatenate([theta, theta], axis=1)       # the two halves of a pair share an angle
+    return qkv, np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def test_rope_is_a_complex_rotation_of_each_pair():
+    """Independent form: pair (x_d, x_{d+D/2}) as x_d + i x_{d+D/2}, multiplied
+    by e^{i theta_d}."""
+    qkv, c, s = _rope_case(7, 3, 16, 120)
+    q, k, v = oracle.qkv_rope(qkv, c, s, oracle.BF16)
+    x = oracle.widen(qkv, oracle.BF16)
+    for src, got in ((x[:, 0], q), (x[:, 1], k)):
+        z = src[..., :8] + 1j * src[..., 8:]
+        e = c[:, None, :8].astype(np.float64) + 1j * s[:, None, :8].astype(np.float64)
+        zr = z * e
+        np.testing.assert_allclose(got[..., :8], zr.real, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(got[..., 8:], zr.imag, rtol=0, atol=1e-12)
+    assert np.array_equal(v, x[:, 2])
+
+
+def test_rope_identity_and_quarter_turn():
+    qkv, _, _ = _rope_case(4, 2, 8, 121, synth.F16)
+    ones, zeros = np.ones((4, 8), np.float32), np.zeros((4, 8), np.float32)
+    x = oracle.widen(qkv, oracle.F16)
+    q, k, _ = oracle.qkv_rope(qkv, ones, zeros, oracle.F16)
+    assert np.array_equal(q, x[:, 0]) and np.array_equal(k, x[:, 1])
+    q, k, _ = oracle.qkv_rope(qkv, zeros, ones, oracle.F16)      # rotate_half itself
+    assert np.array_equal(q[..., :4], -x[:, 0, :, 4:]) and np.array_equal(q[..., 4:], x[:, 0, :, :4])
+
+
+def test_rope_preserves_pair_norms_and_dot_products_shift():
+    qkv, c, s = _rope_case(9, 2, 32, 122)
+    q, k, _ = oracle.qkv_rope(qkv, c, s, oracle.BF16)
+    x = oracle.widen(qkv, oracle.BF16)
+    n0 = x[:, 0, :, :16] ** 2 + x[:, 0, :, 16:] ** 2
+    n1 = q[..., :16] ** 2 + q[..., 16:] ** 2
+    np.testing.assert_allclose(n1, n0, rtol=1e-6)   # cos/sin are float32: |c + i s| = 1 to ~1e-7
+
+
+def test_rope_hand_fixture():
+    # D = 4, one head, one token: q = (1, 2, 3, 4), angle pi/2 on pair 0 and 0 on pair 1
+    qkv = np.zeros((1, 3, 1, 4), np.float64)
+    qkv[0, 0, 0] = [1, 2, 3, 4]
+    qkv[0, 1, 0] = [5, 6, 7, 8]
+    qkv[0, 2, 0] = [9, 10, 11, 12]
+    c = np.array([[0.0, 1.0, 0.0, 1.0]])
+    s = np.array([[1.0, 0.0, 1.0, 0.0]])
+    q, k, v = oracle.qkv_rope(qkv, c, s, oracle.F64)
+    assert q[0, 0].tolist() == [-3.0, 2.0, 1.0, 4.0]
+    assert k[0, 0].tolist() == [-7.0, 6.0, 5.0, 8.0]
+    assert v[0, 0].tolist() == [9.0, 10.0, 11.0, 12.0]
