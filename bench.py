@@ -5,7 +5,10 @@ A step is one call of ``vitattn_forward`` over one batch of the workload:
 the whole path (Q.K^T, online softmax, P.V, epilogue) in one kernel launch.
 For a ragged multi-image workload (``--workload multi_image``) a step is one
 call of ``vitattn_forward_varlen`` over the packed batch, and the flops are
-4*H*D*sum(n_s^2) over its images.
+4*H*D*sum(n_s^2) over its images.  For the prologue workload
+(``--workload rope_batched``) a step is one ``vitattn_qkv_rope`` call (packed
+QKV split + 2-D rope) and the metric is its algorithmic bytes per second
+against the measured HBM copy bandwidth.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
@@ -60,7 +63,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=None,
                     help="timed steps (default: enough for about 2 s of timed work)")
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS) + sorted(synth.RAGGED))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.RAGGED) + sorted(synth.PROLOGUE))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -288,8 +292,178 @@ def run_reference(args):
     return 0
 
 
+PROLOGUE_METRIC = "qkv split + 2-D rope prologue GB/s (algorithmic bytes / device time) and % of measured HBM copy bandwidth"
+
+
+def run_prologue(args):
+    """The prologue workload: one vitattn_qkv_rope call per step."""
+    w = synth.PROLOGUE[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    qkv, cs, sn = synth.make_prologue(w)
+
+    def cpu_leg(seconds, steps=1):
+        # the oracle on a bounded, seeded sample of tokens; bytes scaled per token
+        import oracle
+
+        per_token = w.io_bytes / w.T
+        n, dt = 64, 0.0
+        for attempt in range(8):
+            idx = np.random.Generator(np.random.PCG64(w.seed + attempt)).choice(w.T, min(n, w.T), replace=False)
+            t0 = time.perf_counter()
+            for _ in range(steps):
+                oracle.qkv_rope(qkv[idx], cs[idx], sn[idx], w.dtype)
+            dt = (time.perf_counter() - t0) / steps
+            if dt >= 0.5 * seconds or n >= w.T:
+                break
+            n = int(min(w.T, max(2 * n, n * seconds / max(dt, 1e-6))))
+        return per_token * len(idx) / dt / 1e9, len(idx), dt
+
+    peaks, _ = measured_peaks()
+    peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        import oracle
+
+        value, n, dt = cpu_leg(2.0, steps=max(1, args.steps or 1))
+        line = {"impl": "reference", "metric": PROLOGUE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps or 1, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, "tokens": w.T, "H": w.H, "D": w.D, "sample_tokens": n},
+                "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                                 "sample": f"{n} of {w.T} tokens (seeded), numpy fp64"},
+                "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+
+    from vit_bidirectional_attention_b200 import vitattn
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
+    hqkv = torch.from_numpy(qkv.view(np.int16).copy()).view(tdt)
+    hcs, hsn = torch.from_numpy(cs), torch.from_numpy(sn)
+    dqkv, dcs, dsn = (x.to(dev) for x in (hqkv, hcs, hsn))
+    q, k, v = (torch.empty((w.T, w.H, w.D), dtype=tdt, device=dev) for _ in range(3))
+    stream = torch.cuda.Stream(dev)
+    sh = stream.cuda_stream
+    L = vitattn.lib()
+
+    def step():
+        rc = L.vitattn_qkv_rope(dqkv.data_ptr(), dcs.data_ptr(), dsn.data_ptr(), q.data_ptr(), k.data_ptr(),
+                                v.data_ptr(), w.T, w.H, w.D, w.dtype, sh)
+        if rc:
+            raise vitattn.VitAttnError(rc, "vitattn_qkv_rope")
+
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    sampler.start()
+    warm = 0
+    t_w = time.perf_counter()
+    with torch.cuda.stream(stream):
+        while warm < max(3, args.warmup) or time.perf_counter() - t_w < 1.0:
+            step()
+            warm += 1
+    stream.synchronize()
+    if args.steps is None:
+        w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        w0.record(stream)
+        for _ in range(5):
+            step()
+        w1.record(stream)
+        w1.synchronize()
+        steps = int(max(20, min(20000, 2000.0 / max(w0.elapsed_time(w1) / 5, 1e-3))))
+        steps = int(max_over_ranks(float(steps), world))
+    else:
+        steps = args.steps
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.mark("t_start")
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    ev1.synchronize()
+    sampler.mark("t_stop")
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+    clocks = sampler.stop()
+    ms_step = ms_total / steps
+    gbs = w.io_bytes * steps * world / (ms_total * 1e-3) / 1e9
+    per_gpu = w.io_bytes / (ms_step * 1e-3) / 1e9
+
+    # end to end through the Python entry, host copies on the same stream
+    hqkv_p, hcs_p, hsn_p = (x.pin_memory() for x in (hqkv, hcs, hsn))
+    hq, hk, hv = (torch.empty((w.T, w.H, w.D), dtype=tdt).pin_memory() for _ in range(3))
+
+    def e2e_step():
+        dqkv.copy_(hqkv_p, non_blocking=True)
+        dcs.copy_(hcs_p, non_blocking=True)
+        dsn.copy_(hsn_p, non_blocking=True)
+        oq, ok, ov = vitattn.qkv_rope(dqkv, dcs, dsn, stream=stream)
+        hq.copy_(oq, non_blocking=True)
+        hk.copy_(ok, non_blocking=True)
+        hv.copy_(ov, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            e2e_step()
+    stream.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, args.e2e_steps)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+    e1.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    result = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            import oracle
+
+            value, n, dt = cpu_leg(args.cpu_seconds)
+            cpu = {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                   "sample": f"{n} of {w.T} tokens (seeded), numpy fp64, {dt:.1f} s"}
+        in_bytes = 3 * w.T * w.H * w.D * 2 + 2 * w.T * w.D * 4
+        result = {
+            "metric": PROLOGUE_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": synth.DTYPE_NAMES[w.dtype],
+            "data": "synthetic (seeded normals; 2-D rope tables of the patch grid)",
+            "config": {"workload": w.name, "images": w.images, "grid": list(w.grid), "tokens": w.T, "H": w.H,
+                       "D": w.D, "global_batch": w.images * world,
+                       "l2": f"{w.io_bytes / 2**20:.0f} MiB moved per step > 126 MiB L2, no flush",
+                       "bytes_per_step": w.io_bytes},
+            "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s", "frac": per_gpu / peak,
+                         "traffic": committed_traffic(w.name),
+                         "peak_source": "measured copy bandwidth, MEASURED_PEAKS.json" if peaks else "fallback",
+                         "kernel": "vitattn::qkv_rope_kernel", "algorithmic_bytes_per_launch": w.io_bytes},
+            "e2e": {"value": w.io_bytes * n_e2e * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": 3 * w.T * w.H * w.D * 2,
+                    "ms_per_step": e2e_ms / n_e2e, "entry": "qkv_rope + stream copies"},
+            "gpu_launches": steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+    ranks.finish(world)
+    if result is not None:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload in synth.PROLOGUE:
+        return run_prologue(args)
     if args.impl == "reference":
         return run_reference(args)
     import numpy as np

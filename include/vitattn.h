@@ -160,6 +160,38 @@ VITATTN_API int vitattn_check_args_varlen(const void* q, const void* k, const vo
                                           float scale, int dtype);
 
 /*
+ * vitattn_qkv_rope -- the attention's prologue: split a packed QKV projection
+ * into q, k, v and apply the rotary embedding to q and k, in one pass.
+ * Source: inferencelayer "src/vision_gpu.rs", VIS_QKV_ROPE and its doc (the
+ * projection output is q | k | v per token; the rope tables arrive
+ * precomputed, so a 2-D rope is whatever row/column walk built them;
+ * rotate_half pairs element d with d +- D/2, negated on the low half; v is
+ * not rotated).
+ *   qkv       device pointer, [T, 3, H, D] of `dtype` (token-major: each
+ *             token's q heads, then its k heads, then its v heads).
+ *   cos_table, sin_table  device pointers, [T, D] float32, one row per token
+ *             (shared by every head).
+ *   q, k, v   device pointers, [T, H, D] of `dtype`: the layout the
+ *             attention entries read (T = B*N dense, or the ragged total).
+ *             They must not overlap each other or the inputs.
+ *   T, H      tokens and heads (>= 1); D as for vitattn_forward (16..128,
+ *             D % 8 == 0).  All pointers 16-byte aligned.
+ * Per token t, head h, and x = q or k:
+ *     x'[d] = x[d] * cos[t,d] + r[d] * sin[t,d],
+ *     r[d]  = -x[d + D/2] (d < D/2),  x[d - D/2] (d >= D/2),
+ * computed in f32 and rounded once to `dtype`; v is copied bit for bit.
+ * Enqueues one kernel on `stream`; errors as for vitattn_forward.
+ */
+VITATTN_API int vitattn_qkv_rope(const void* qkv, const float* cos_table, const float* sin_table, void* q,
+                                 void* k, void* v, int64_t T, int64_t H, int64_t D, int dtype,
+                                 vitattn_stream_t stream);
+
+/* The argument checks of vitattn_qkv_rope alone (no CUDA call). */
+VITATTN_API int vitattn_check_args_qkv_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                                            const void* q, const void* k, const void* v, int64_t T, int64_t H,
+                                            int64_t D, int dtype);
+
+/*
  * vitattn_forward_host -- the same operation from HOST buffers: enqueues the
  * copies hq->dq, hk->dk, hv->dv, the kernel, and dout->hout, in that order,
  * on `stream`, and returns without synchronising.  The caller synchronises

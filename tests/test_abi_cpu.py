@@ -134,3 +134,34 @@ def test_varlen_argument_errors(kw, code):
 def test_varlen_with_no_tokens_is_a_no_op_without_cuda():
     assert vitattn.forward_varlen_ptr(Q, K, V, O, [0, 0, 0], 2, 64, 0.125, vitattn.BF16) == 0
     assert vitattn.forward_varlen_ptr(Q, K, V, O, [0, 5, 3], 2, 64, 0.125, vitattn.BF16) == -12
+
+
+# ---------------------------------------------------------------- QKV split + rope prologue
+
+def check_rope(**kw):
+    T, H, D = kw.get("T", 64), kw.get("H", 2), kw.get("D", 64)
+    row = max(H * D * 2, 16)
+    # disjoint fake regions: qkv | cos | sin | q | k | v
+    a = dict(qkv=A, cos=A + 3 * row * T, sin=A + 3 * row * T + T * D * 4, q=A + 3 * row * T + 2 * T * D * 4,
+             T=T, H=H, D=D, dtype=vitattn.BF16)
+    a["k"] = a["q"] + row * T
+    a["v"] = a["k"] + row * T
+    a.update(kw)
+    return vitattn.check_args_qkv_rope(a["qkv"], a["cos"], a["sin"], a["q"], a["k"], a["v"], a["T"], a["H"], a["D"],
+                                       a["dtype"])
+
+
+def test_rope_valid_arguments_pass():
+    assert check_rope() == 0
+    assert check_rope(D=128, dtype=vitattn.F16) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(qkv=0), -1), (dict(sin=0), -1), (dict(v=0), -1),
+    (dict(T=0), -2), (dict(H=0), -2), (dict(D=60), -3), (dict(D=8), -3), (dict(D=136), -3), (dict(dtype=5), -4),
+    (dict(cos=A + 3 * 256 * 64 + 4), -5),
+    (dict(q=A + 16), -6),                       # inside qkv
+    (dict(k=A + 3 * 256 * 64 + 16), -6),        # inside the cos table
+])
+def test_rope_argument_errors(kw, code):
+    assert check_rope(**kw) == code

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -13,6 +14,7 @@
 #include "vitattn.h"
 
 #include "fwd_kernel.cuh"
+#include "rope_kernel.cuh"
 
 namespace {
 
@@ -35,6 +37,12 @@ int cuda_fail(cudaError_t e) {
 bool overlaps(const void* a, const void* b, uint64_t bytes) {
     const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
     return x < y + bytes && y < x + bytes;
+}
+
+// [a, a + la) and [b, b + lb) share a byte.
+bool overlaps2(const void* a, uint64_t la, const void* b, uint64_t lb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + lb && y < x + la;
 }
 
 int check_args(const void* q, const void* k, const void* v, const void* out, int64_t B, int64_t N,
@@ -90,6 +98,33 @@ int check_args_varlen(const void* q, const void* k, const void* v, const void* o
     const uint64_t bytes = token_bytes * (uint64_t)total;
     if (bytes > 0 && (overlaps(out, q, bytes) || overlaps(out, k, bytes) || overlaps(out, v, bytes)))
         return VITATTN_ERR_ALIAS;
+    return VITATTN_OK;
+}
+
+// QKV split + rope prologue: qkv [T, 3, H, D], cos/sin [T, D] f32, q/k/v [T, H, D].
+int check_args_rope(const void* qkv, const float* cs, const float* sn, const void* q, const void* k,
+                    const void* v, int64_t T, int64_t H, int64_t D, int dtype) {
+    if (!qkv || !cs || !sn || !q || !k || !v) return VITATTN_ERR_NULL;
+    if (T < 1 || H < 1 || D < 1) return VITATTN_ERR_DIM;
+    if (D < 16 || D > 128 || D % 8 != 0) return VITATTN_ERR_HEADDIM;
+    if (dtype != VITATTN_BF16 && dtype != VITATTN_F16) return VITATTN_ERR_DTYPE;
+    if (H > (int64_t)INT32_MAX || T > (int64_t)1 << 40) return VITATTN_ERR_DIM;
+    const uint64_t row_bytes = (uint64_t)H * (uint64_t)D * 2u;
+    if (row_bytes >= (1ull << 40) || (uint64_t)T > (1ull << 60) / (3u * row_bytes)) return VITATTN_ERR_DIM;
+    const uintptr_t mis = (reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(cs) |
+                           reinterpret_cast<uintptr_t>(sn) | reinterpret_cast<uintptr_t>(q) |
+                           reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15u;
+    if (mis) return VITATTN_ERR_ALIGN;
+    const uint64_t in_bytes = 3u * row_bytes * (uint64_t)T, out_bytes = row_bytes * (uint64_t)T;
+    const uint64_t tab_bytes = (uint64_t)T * (uint64_t)D * 4u;
+    const void* outs[3] = {q, k, v};
+    for (int i = 0; i < 3; ++i) {
+        if (overlaps2(outs[i], out_bytes, qkv, in_bytes) || overlaps2(outs[i], out_bytes, cs, tab_bytes) ||
+            overlaps2(outs[i], out_bytes, sn, tab_bytes))
+            return VITATTN_ERR_ALIAS;
+        for (int j = 0; j < i; ++j)
+            if (overlaps(outs[i], outs[j], out_bytes)) return VITATTN_ERR_ALIAS;
+    }
     return VITATTN_OK;
 }
 
@@ -332,6 +367,31 @@ int launch_varlen(const void* q, const void* k, const void* v, void* out, const 
     return run_kernel(dp, dtype, kModeVarlen, (unsigned)items, &prm, &seg, stream);
 }
 
+// The prologue: a grid-stride kernel, 8 warps per block, at most 8 blocks per SM
+// (a full SM), one warp per (token, head).
+int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void* k, void* v, int64_t T,
+                int64_t H, int64_t D, int dtype, cudaStream_t stream) {
+    int rc = check_args_rope(qkv, cs, sn, q, k, v, T, H, D, dtype);
+    if (rc) return rc;
+    int num_sms = 0;
+    rc = device_info(&num_sms);
+    if (rc) return rc;
+    const uint64_t items = (uint64_t)T * (uint64_t)((H + vitattn::kRopeHeadsPerWarp - 1) / vitattn::kRopeHeadsPerWarp);
+    const uint64_t per_block = (uint64_t)(vitattn::kRopeThreads / 32);
+    const uint64_t want = (items + per_block - 1) / per_block;
+    const unsigned grid = (unsigned)std::min<uint64_t>(want, (uint64_t)num_sms * 8u);
+    auto qkv8 = static_cast<const uint8_t*>(qkv);
+    auto q8 = static_cast<uint8_t*>(q), k8 = static_cast<uint8_t*>(k), v8 = static_cast<uint8_t*>(v);
+    long long TT = (long long)T;
+    int HH = (int)H, DD = (int)D;
+    void* args[9] = {&qkv8, &cs, &sn, &q8, &k8, &v8, &TT, &HH, &DD};
+    const void* fn = dtype == VITATTN_BF16 ? reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true>)
+                                           : reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false>);
+    cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(vitattn::kRopeThreads), args, 0, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return VITATTN_OK;
+}
+
 // Launch (through `go`), synchronise, and read the kernel's status words.
 template <class Go>
 int checked_run(cudaStream_t stream, Go go) {
@@ -428,6 +488,16 @@ int vitattn_check_args_varlen(const void* q, const void* k, const void* v, const
                               const int32_t* cu_seqlens, int64_t num_seqs, int64_t H, int64_t D,
                               float scale, int dtype) {
     return check_args_varlen(q, k, v, out, cu_seqlens, num_seqs, H, D, scale, dtype);
+}
+
+int vitattn_qkv_rope(const void* qkv, const float* cos_table, const float* sin_table, void* q, void* k, void* v,
+                     int64_t T, int64_t H, int64_t D, int dtype, vitattn_stream_t stream) {
+    return launch_rope(qkv, cos_table, sin_table, q, k, v, T, H, D, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int vitattn_check_args_qkv_rope(const void* qkv, const float* cos_table, const float* sin_table, const void* q,
+                                const void* k, const void* v, int64_t T, int64_t H, int64_t D, int dtype) {
+    return check_args_rope(qkv, cos_table, sin_table, q, k, v, T, H, D, dtype);
 }
 
 int vitattn_forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq,

@@ -31,6 +31,12 @@ with ``cu_seqlens`` start offsets, each image attending only within itself):
   inputs and output, more than the 126 MiB L2), 16 heads, D = 80, bf16,
   Q,K iid N(0, 1.5^2), V iid N(0,1) (the ``doc_page`` distribution).
 
+The attention's prologue (packed QKV split + 2-D rope, ``[T, 3, H, D]`` in):
+
+- ``rope_batched``  the QKV of ``batched``: 32 images of 32 x 32 patches
+  (32 768 tokens), 16 heads, D = 64, bf16, iid N(0,1), with the 2-D rope
+  tables of a 32 x 32 patch grid (``rope_tables_2d``) repeated per image.
+
 Every workload uses scale = 1/sqrt(D) and seed 20261202 + its index.
 """
 from __future__ import annotations
@@ -163,6 +169,75 @@ def random_ragged(seqlens, H: int, D: int, dtype: int, seed: int, std: float = 1
     w = RaggedWorkload("sweep", tuple(int(n) for n in seqlens), H, D, dtype, qk_std=std)
     q, k, v = make_qkv_ragged(w, seed=seed)
     return q, k, v, w.cu_seqlens
+
+
+def rope_tables_2d(grid_h: int, grid_w: int, D: int, theta: float = 10000.0):
+    """cos, sin ``[grid_h*grid_w, D]`` float32 for the patches of an h x w grid
+    in row-major order: a 2-D rotary embedding whose first D/4 frequency pairs
+    turn with the patch row and the next D/4 with the patch column, each
+    angle shared by the pair (d, d + D/2) that ``rotate_half`` rotates.
+    (These are the kernel's inputs, built the way the pages say the CPU
+    tower builds them: a (row, col) walk, with the rotation applied
+    elsewhere.)"""
+    quarter = D // 4
+    inv_freq = theta ** (-np.arange(quarter, dtype=np.float64) / quarter)
+    r, c = np.divmod(np.arange(grid_h * grid_w, dtype=np.float64), grid_w)
+    ang = np.concatenate([r[:, None] * inv_freq[None, :], c[:, None] * inv_freq[None, :]], axis=1)
+    if ang.shape[1] < D // 2:  # D/2 odd: the last pair gets angle 0
+        ang = np.concatenate([ang, np.zeros((ang.shape[0], D // 2 - ang.shape[1]))], axis=1)
+    ang = np.concatenate([ang, ang], axis=1)
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+@dataclasses.dataclass(frozen=True)
+class PrologueWorkload:
+    """A packed QKV projection of ``images`` images of ``grid`` patches each,
+    with their 2-D rope tables: the input of the QKV split + rope prologue."""
+    name: str
+    images: int
+    grid: tuple
+    H: int
+    D: int
+    dtype: int
+    index: int = 0
+
+    @property
+    def seed(self) -> int:
+        return SEED_BASE + self.index
+
+    @property
+    def T(self) -> int:
+        return self.images * self.grid[0] * self.grid[1]
+
+    @property
+    def io_bytes(self) -> int:
+        """qkv read, cos/sin read, q/k/v written: each once."""
+        return 2 * (3 * self.T * self.H * self.D * 2) + 2 * self.T * self.D * 4
+
+
+PROLOGUE = {
+    w.name: w
+    for w in (
+        # the QKV of the batched workload: 32 images of 32 x 32 patches, 16 heads, D = 64
+        PrologueWorkload("rope_batched", 32, (32, 32), 16, 64, BF16, index=6),
+    )
+}
+
+
+def make_prologue(w: PrologueWorkload):
+    """(qkv bits [T, 3, H, D], cos [T, D], sin [T, D]) for prologue workload ``w``."""
+    qkv = make_qkv_packed(w.T, w.H, w.D, w.dtype, seed=w.seed)
+    cs, sn = rope_tables_2d(w.grid[0], w.grid[1], w.D)
+    return qkv, np.tile(cs, (w.images, 1)), np.tile(sn, (w.images, 1))
+
+
+def make_qkv_packed(T: int, H: int, D: int, dtype: int, seed: int, std: float = 1.0):
+    """A packed QKV projection output ``[T, 3, H, D]`` (bit patterns), iid N(0, std^2)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = rng.standard_normal(size=(T, 3, H, D), dtype=np.float32)
+    if std != 1.0:
+        x *= np.float32(std)
+    return round_to_bits(x, dtype)
 
 
 def round_to_bits(x: np.ndarray, dtype: int) -> np.ndarray:

@@ -62,13 +62,16 @@ def lib() -> ctypes.CDLL:
         L.vitattn_forward_varlen_checked.argtypes = var
         L.vitattn_test_forward_varlen_flags.argtypes = var + [i32]
         L.vitattn_check_args_varlen.argtypes = var[:-1]
+        rope = [p, p, p, p, p, p, i64, i64, i64, i32]
+        L.vitattn_qkv_rope.argtypes = rope + [p]
+        L.vitattn_check_args_qkv_rope.argtypes = rope
         L.vitattn_strerror.argtypes = [i32]
         L.vitattn_strerror.restype = ctypes.c_char_p
         for f in (L.vitattn_forward, L.vitattn_forward_checked, L.vitattn_test_forward_flags,
                   L.vitattn_forward_host, L.vitattn_check_args, L.vitattn_last_cuda_error,
                   L.vitattn_version, L.vitattn_launches_per_call, L.vitattn_forward_varlen,
                   L.vitattn_forward_varlen_checked, L.vitattn_test_forward_varlen_flags,
-                  L.vitattn_check_args_varlen):
+                  L.vitattn_check_args_varlen, L.vitattn_qkv_rope, L.vitattn_check_args_qkv_rope):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -226,3 +229,51 @@ def forward_varlen(q, k, v, cu_seqlens, out=None, scale=None, stream=None, check
     if rc != 0:
         raise VitAttnError(rc, "vitattn_forward_varlen")
     return out
+
+
+def check_args_qkv_rope(qkv, cos, sin, q, k, v, T, H, D, dtype) -> int:
+    """Status the prologue's argument checks give (pointers as ints); no CUDA call."""
+    return int(lib().vitattn_check_args_qkv_rope(qkv, cos, sin, q, k, v, T, H, D, dtype))
+
+
+def qkv_rope_ptr(qkv, cos, sin, q, k, v, T, H, D, dtype, stream=0) -> int:
+    """Raw prologue call on device pointers (ints); returns the status."""
+    return int(lib().vitattn_qkv_rope(qkv, cos, sin, q, k, v, T, H, D, dtype, stream))
+
+
+def qkv_rope(qkv, cos, sin, stream=None):
+    """Split a packed QKV projection and rotate q and k on CUDA tensors.
+
+    qkv: contiguous ``[..., 3, H, D]`` bf16 / f16 (``[T, 3, H, D]`` or
+    ``[B, N, 3, H, D]``); cos, sin: contiguous float32 ``[T, D]`` (one row
+    per token, T = the product of the leading dims).  Returns (q, k, v), each
+    ``[..., H, D]`` (the attention entries' layout).
+    """
+    import torch
+
+    if qkv.dim() < 4 or qkv.shape[-3] != 3:
+        raise ValueError("qkv must be [..., 3, H, D]")
+    if not (qkv.is_cuda and cos.is_cuda and sin.is_cuda):
+        raise ValueError("qkv, cos, sin must be CUDA tensors")
+    if not (qkv.is_contiguous() and cos.is_contiguous() and sin.is_contiguous()):
+        raise ValueError("qkv, cos, sin must be contiguous")
+    if cos.dtype != torch.float32 or sin.dtype != torch.float32:
+        raise TypeError("cos and sin must be float32")
+    dtype = _dtype_code(qkv)
+    lead = tuple(qkv.shape[:-3])
+    H, D = qkv.shape[-2], qkv.shape[-1]
+    T = 1
+    for n in lead:
+        T *= n
+    if tuple(cos.shape) != (T, D) or tuple(sin.shape) != (T, D):
+        raise ValueError("cos and sin must be [T, D] with T the token count of qkv")
+    q, k, v = (torch.empty(lead + (H, D), dtype=qkv.dtype, device=qkv.device) for _ in range(3))
+    if stream is None:
+        stream = torch.cuda.current_stream(qkv.device)
+    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    with torch.cuda.device(qkv.device):
+        rc = qkv_rope_ptr(qkv.data_ptr(), cos.data_ptr(), sin.data_ptr(), q.data_ptr(), k.data_ptr(),
+                          v.data_ptr(), T, H, D, dtype, handle)
+    if rc != 0:
+        raise VitAttnError(rc, "vitattn_qkv_rope")
+    return q, k, v
