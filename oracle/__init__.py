@@ -115,6 +115,21 @@ def probs(q, k, scale: float, dtype: int, b: int, h: int) -> np.ndarray:
     return P
 
 
+def attention_gqa(q, k, v, scale: float, dtype: int, mode: int = MODE_TWO_PASS) -> np.ndarray:
+    """Grouped-query attention: ``q`` is ``[B, N, H, D]``, ``k`` and ``v`` are
+    ``[B, N, Hkv, D]`` with ``H`` a multiple of ``Hkv``; query head ``h``
+    attends with key/value head ``h // (H // Hkv)`` (hf2q
+    ``src/inference/vision/vit_gpu.rs``, doc of ``vit_repeat_kv_gpu``: each
+    kv head is replicated ``num_kv_groups`` times, output row ``h`` reading
+    kv head ``h / num_kv_groups``).  Written as that replication followed by
+    the plain attention."""
+    H, Hkv = q.shape[2], k.shape[2]
+    if Hkv < 1 or H % Hkv or v.shape != k.shape or k.shape[:2] != q.shape[:2] or k.shape[3] != q.shape[3]:
+        raise ValueError("k, v must be [B, N, Hkv, D] with H a multiple of Hkv")
+    g = H // Hkv
+    return attention(q, np.repeat(k, g, axis=2), np.repeat(v, g, axis=2), scale, dtype, mode)
+
+
 def attention_varlen(q, k, v, cu_seqlens, scale: float, dtype: int, mode: int = MODE_TWO_PASS) -> np.ndarray:
     """Ragged batch of images packed along the token axis: ``q, k, v`` are
     ``[total, H, D]`` and segment s covers tokens ``cu_seqlens[s] ..

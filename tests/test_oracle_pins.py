@@ -424,3 +424,40 @@ def test_rope_hand_fixture():
     assert q[0, 0].tolist() == [-3.0, 2.0, 1.0, 4.0]
     assert k[0, 0].tolist() == [-7.0, 6.0, 5.0, 8.0]
     assert v[0, 0].tolist() == [9.0, 10.0, 11.0, 12.0]
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (6, 3), (4, 1), (3, 3)])
+def test_gqa_oracle_matches_per_head_brute_force(H, Hkv):
+    """Independent form: per (b, h) softmax over keys of kv head h // (H/Hkv)."""
+    B, N, D = 2, 5, 8
+    q = synth.round_to_bits(rnd((B, N, H, D), 130).astype(np.float32), synth.BF16)
+    k = synth.round_to_bits(rnd((B, N, Hkv, D), 131).astype(np.float32), synth.BF16)
+    v = synth.round_to_bits(rnd((B, N, Hkv, D), 132).astype(np.float32), synth.BF16)
+    got = oracle.attention_gqa(q, k, v, 0.35, oracle.BF16)
+    qf, kf, vf = (oracle.widen(x, oracle.BF16) for x in (q, k, v))
+    g = H // Hkv
+    for b in range(B):
+        for h in range(H):
+            s = 0.35 * qf[b, :, h] @ kf[b, :, h // g].T
+            w = np.exp(s - s.max(axis=1, keepdims=True))
+            w /= w.sum(axis=1, keepdims=True)
+            np.testing.assert_allclose(got[b, :, h], w @ vf[b, :, h // g], rtol=0, atol=1e-12)
+
+
+def test_gqa_oracle_heads_of_a_group_share_keys_and_values():
+    q1 = synth.round_to_bits(rnd((1, 6, 1, 8), 133).astype(np.float32), synth.F16)
+    q = np.concatenate([q1, q1, q1, q1], axis=2)          # 4 identical query heads
+    k = synth.round_to_bits(rnd((1, 6, 2, 8), 134).astype(np.float32), synth.F16)
+    v = synth.round_to_bits(rnd((1, 6, 2, 8), 135).astype(np.float32), synth.F16)
+    o = oracle.attention_gqa(q, k, v, 0.5, oracle.F16)
+    assert np.array_equal(o[:, :, 0], o[:, :, 1]) and np.array_equal(o[:, :, 2], o[:, :, 3])
+    assert not np.array_equal(o[:, :, 0], o[:, :, 2])
+
+
+def test_gqa_oracle_rejects_bad_head_counts():
+    q = np.zeros((1, 2, 6, 8), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.attention_gqa(q, np.zeros((1, 2, 4, 8), np.uint16), np.zeros((1, 2, 4, 8), np.uint16), 1.0,
+                             oracle.BF16)
