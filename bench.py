@@ -173,6 +173,10 @@ def oracle_rows(w, q, k, v, rows):
     """The oracle on sampled output rows; returns the flops those rows cost."""
     import oracle
 
+    if isinstance(w, synth.Workload) and w.Hkv:
+        g = w.H // w.Hkv
+        oracle.attention_rows(q, np.repeat(k, g, axis=2), np.repeat(v, g, axis=2), w.scale, w.dtype, rows)
+        return 4.0 * w.N * w.D * len(rows)
     if isinstance(w, synth.RaggedWorkload):
         oracle.attention_varlen_rows(q, k, v, w.cu_seqlens, w.scale, w.dtype, rows)
         seg_len = np.diff(np.asarray(w.cu_seqlens))
@@ -245,7 +249,10 @@ def shape_config(w):
     if isinstance(w, synth.RaggedWorkload):
         return {"images": len(w.seqlens), "seqlens": list(w.seqlens), "total_tokens": w.total,
                 "H": w.H, "D": w.D}
-    return {"B": w.B, "N": w.N, "H": w.H, "D": w.D}
+    cfg = {"B": w.B, "N": w.N, "H": w.H, "D": w.D}
+    if w.Hkv:
+        cfg["Hkv"] = w.Hkv
+    return cfg
 
 
 def run_reference(args):
@@ -474,6 +481,7 @@ def main():
     world, rank, local = dist_setup(args)
     w, q, k, v = load_workload(args.workload)
     ragged = isinstance(w, synth.RaggedWorkload)
+    gqa = not ragged and bool(w.Hkv)
     tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
     dev = torch.device("cuda", local if world > 1 else 0)
 
@@ -482,7 +490,7 @@ def main():
 
     hq, hk, hv = (host(x) for x in (q, k, v))
     dq, dk, dv = (x.to(dev) for x in (hq, hk, hv))
-    dout = torch.empty_like(dq)
+    dout = torch.empty_like(dq)  # [.., H, D] like q (k, v may have fewer heads)
     stream = torch.cuda.Stream(dev)
     sh = stream.cuda_stream
     L = vitattn.lib()
@@ -498,6 +506,12 @@ def main():
                                           n_seqs, w.H, w.D, w.scale, w.dtype, sh)
             if rc:
                 raise vitattn.VitAttnError(rc, "vitattn_forward_varlen")
+    elif gqa:
+        def step():
+            rc = L.vitattn_forward_gqa(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B, w.N,
+                                       w.H, w.Hkv, w.D, w.scale, w.dtype, sh)
+            if rc:
+                raise vitattn.VitAttnError(rc, "vitattn_forward_gqa")
     else:
         def step():
             rc = L.vitattn_forward(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
@@ -510,6 +524,9 @@ def main():
         if ragged:
             rc = vitattn.forward_varlen_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(),
                                             w.cu_seqlens, w.H, w.D, w.scale, w.dtype, sh, checked=True)
+        elif gqa:
+            rc = vitattn.forward_gqa_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B, w.N,
+                                         w.H, w.Hkv, w.D, w.scale, w.dtype, sh, checked=True)
         else:
             rc = vitattn.forward_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
                                      w.N, w.H, w.D, w.scale, w.dtype, sh, checked=True)
@@ -560,14 +577,17 @@ def main():
 
     # end to end through the host-buffer entry point
     hq_p, hk_p, hv_p = (x.pin_memory() for x in (hq, hk, hv))
-    hout_p = torch.empty_like(hq).pin_memory()
+    hout_p = torch.empty_like(hq).pin_memory()  # like q
     e2e_steps = max(1, args.e2e_steps)
 
-    if ragged:
+    if ragged or gqa:
         def e2e_step():
             for d, h in ((dq, hq_p), (dk, hk_p), (dv, hv_p)):
                 d.copy_(h, non_blocking=True)
-            vitattn.forward_varlen(dq, dk, dv, w.cu_seqlens, out=dout, scale=w.scale, stream=stream)
+            if ragged:
+                vitattn.forward_varlen(dq, dk, dv, w.cu_seqlens, out=dout, scale=w.scale, stream=stream)
+            else:
+                vitattn.forward_gqa(dq, dk, dv, out=dout, scale=w.scale, stream=stream)
             hout_p.copy_(dout, non_blocking=True)
     else:
         def e2e_step():
@@ -644,9 +664,11 @@ def main():
                 "achieved_hbm_gbs": w.io_bytes / (ms_step * 1e-3) / 1e9,
             },
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": 3 * w.numel * 2, "d2h_bytes_per_step": w.numel * 2,
+                    "h2d_bytes_per_step": sum(x.numel() for x in (hq, hk, hv)) * 2,
+                    "d2h_bytes_per_step": hq.numel() * 2,
                     "ms_per_step": e2e_ms / e2e_steps,
-                    "entry": "forward_varlen + stream copies" if ragged else "vitattn_forward_host"},
+                    "entry": ("forward_varlen + stream copies" if ragged else
+                              "forward_gqa + stream copies" if gqa else "vitattn_forward_host")},
             "gpu_launches": args.steps * vitattn.launches_per_call(),
             "clocks": clocks,
             "cpu_baseline": cpu,

@@ -116,6 +116,30 @@ VITATTN_API int vitattn_forward_checked(const void* q, const void* k, const void
                             int64_t N, int64_t H, int64_t D, float scale, int dtype,
                             vitattn_stream_t stream);
 
+/*
+ * vitattn_forward_gqa -- grouped-query attention: H query heads share Hkv
+ * key/value heads, query head h using key/value head h / (H / Hkv).
+ * Source: hf2q "src/inference/vision/vit_gpu.rs", doc of `vit_repeat_kv_gpu`
+ * (each kv head replicated num_kv_groups times; output row h reads kv head
+ * h / num_kv_groups).  No replicated copy is made: each CTA reads its kv
+ * head directly.
+ *   q, out    [B, N, H, D];  k, v  [B, N, Hkv, D];  1 <= Hkv, H % Hkv == 0
+ *             (VITATTN_ERR_DIM otherwise).  Everything else as for
+ *             vitattn_forward (Hkv = H is exactly vitattn_forward).
+ */
+VITATTN_API int vitattn_forward_gqa(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
+                                    int64_t H, int64_t Hkv, int64_t D, float scale, int dtype,
+                                    vitattn_stream_t stream);
+
+/* vitattn_forward_gqa, then a stream synchronisation and a read of the kernel's status words. */
+VITATTN_API int vitattn_forward_gqa_checked(const void* q, const void* k, const void* v, void* out, int64_t B,
+                                            int64_t N, int64_t H, int64_t Hkv, int64_t D, float scale, int dtype,
+                                            vitattn_stream_t stream);
+
+/* The argument checks of vitattn_forward_gqa alone (no CUDA call). */
+VITATTN_API int vitattn_check_args_gqa(const void* q, const void* k, const void* v, const void* out, int64_t B,
+                                       int64_t N, int64_t H, int64_t Hkv, int64_t D, float scale, int dtype);
+
 /* Most segments one vitattn_forward_varlen call takes. */
 #define VITATTN_MAX_SEQS 256
 

@@ -165,3 +165,25 @@ def test_rope_valid_arguments_pass():
 ])
 def test_rope_argument_errors(kw, code):
     assert check_rope(**kw) == code
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+def check_gqa(**kw):
+    a = dict(q=Q, k=K, v=V, out=O, B=1, N=64, H=2, Hkv=1, D=64, scale=0.125, dtype=vitattn.BF16)
+    a.update(kw)
+    return vitattn.check_args_gqa(a["q"], a["k"], a["v"], a["out"], a["B"], a["N"], a["H"], a["Hkv"], a["D"],
+                                  a["scale"], a["dtype"])
+
+
+def test_gqa_valid_arguments_pass():
+    assert check_gqa() == 0
+    assert check_gqa(Hkv=2) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), -1), (dict(q=0), -1), (dict(Hkv=0), -2), (dict(H=3, Hkv=2), -2), (dict(Hkv=4), -2),
+    (dict(D=70), -3), (dict(dtype=7), -4), (dict(v=V + 4), -5), (dict(out=K + 16), -6), (dict(out=Q), -6),
+])
+def test_gqa_argument_errors(kw, code):
+    assert check_gqa(**kw) == code

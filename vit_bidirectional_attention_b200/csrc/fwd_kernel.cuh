@@ -202,6 +202,7 @@ struct alignas(64) FwdParams {
     int n_qgroups;      // ceil(N / (128 * tiles_per_cta)): work items per (b, h) (dense layout)
     int n_items;        // all work items; a CTA takes items blockIdx.x + k * gridDim.x
     int n_kblocks;      // ceil(N / 128) (dense layout; a ragged batch takes it per segment)
+    int kv_group;       // query heads per key/value head (1: multi-head; H / Hkv: grouped-query)
     float scale_log2;
     int flags;
     unsigned long long timeout_ns;
@@ -647,8 +648,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                         for (int c = 0; c < NCH; ++c)
                             ptx::tma_load_4d(sKV + slot * TILE + 256 * chunk_col(DP, c),
                                              &p.maps[1 + kv][width_class(chunk_width(DP, c))],
-                                             chunk_col(DP, c), it.h, it.tok0 + j * kBlockKeys, it.b,
-                                             bar(kBarKvFull + slot));
+                                             chunk_col(DP, c), it.h / p.kv_group, it.tok0 + j * kBlockKeys,
+                                             it.b, bar(kBarKvFull + slot));
                     }
                 }
             }

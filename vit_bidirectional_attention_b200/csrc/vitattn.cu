@@ -70,6 +70,22 @@ int check_args(const void* q, const void* k, const void* v, const void* out, int
     return VITATTN_OK;
 }
 
+// Grouped-query attention: q, out [B, N, H, D]; k, v [B, N, Hkv, D], H a multiple of Hkv.
+int check_args_gqa(const void* q, const void* k, const void* v, const void* out, int64_t B, int64_t N,
+                   int64_t H, int64_t Hkv, int64_t D, float scale, int dtype) {
+    if (Hkv < 1 || H < 1 || H % Hkv != 0) return (!q || !k || !v || !out) ? VITATTN_ERR_NULL : VITATTN_ERR_DIM;
+    // the query side (and every shape limit) as for multi-head attention, with k, v
+    // standing in at the query's size only for the pointer checks
+    int rc = check_args(q, q, q, out, B, N, H, D, scale, dtype);
+    if (rc) return rc;
+    if (!k || !v) return VITATTN_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15u) return VITATTN_ERR_ALIGN;
+    const uint64_t out_bytes = (uint64_t)B * (uint64_t)N * (uint64_t)H * (uint64_t)D * 2u;
+    const uint64_t kv_bytes = (uint64_t)B * (uint64_t)N * (uint64_t)Hkv * (uint64_t)D * 2u;
+    if (overlaps2(out, out_bytes, k, kv_bytes) || overlaps2(out, out_bytes, v, kv_bytes)) return VITATTN_ERR_ALIAS;
+    return VITATTN_OK;
+}
+
 // Ragged batch: q, k, v, out are [total, H, D] with total = cu_seqlens[num_seqs];
 // cu_seqlens (host) starts at 0 and never decreases.
 int check_args_varlen(const void* q, const void* k, const void* v, const void* out,
@@ -254,18 +270,21 @@ int ensure_smem(int dp, int dtype, Mode mode, const void* fn) {
 
 // Tensor maps of q, k, v for every column-chunk width, and the shape fields.
 int fill_common(FwdParams* prm, const void* q, const void* k, const void* v, void* out, int64_t B,
-                int64_t N, int64_t H, int64_t D, float scale, int dtype, int flags) {
+                int64_t N, int64_t H, int64_t D, float scale, int dtype, int flags, int64_t Hkv = 0) {
     std::memset(prm, 0, sizeof *prm);
+    if (Hkv == 0) Hkv = H;  // multi-head: k and v have the query's head count
     const int dp = (int)((D + 15) / 16 * 16);
     const void* src[3] = {q, k, v};
+    const int64_t heads[3] = {H, Hkv, Hkv};
     const int nch = vitattn::chunk_count(dp);
     for (int c = 0; c < nch; ++c) {
         const int w = vitattn::chunk_width(dp, c);
         for (int m = 0; m < 3; ++m) {
             CUtensorMap* map = &prm->maps[m][vitattn::width_class(w)];
-            if (!encode_map(map, src[m], dtype, B, N, H, D, w)) return cuda_fail(cudaErrorInvalidValue);
+            if (!encode_map(map, src[m], dtype, B, N, heads[m], D, w)) return cuda_fail(cudaErrorInvalidValue);
         }
     }
+    prm->kv_group = (int)(H / Hkv);
     prm->out = out;
     prm->B = (int)B;
     prm->N = (int)N;
@@ -292,8 +311,9 @@ int run_kernel(int dp, int dtype, Mode mode, unsigned grid, FwdParams* prm, Seg*
 }
 
 int launch(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
-           int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags) {
-    int rc = check_args(q, k, v, out, B, N, H, D, scale, dtype);
+           int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags, int64_t Hkv = 0) {
+    int rc = Hkv ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
+                 : check_args(q, k, v, out, B, N, H, D, scale, dtype);
     if (rc) return rc;
     const int dp = (int)((D + 15) / 16 * 16);
     int num_sms = 0;
@@ -301,7 +321,7 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     if (rc) return rc;
 
     FwdParams prm;
-    rc = fill_common(&prm, q, k, v, out, B, N, H, D, scale, dtype, flags);
+    rc = fill_common(&prm, q, k, v, out, B, N, H, D, scale, dtype, flags, Hkv);
     if (rc) return rc;
     // Two query tiles per CTA share each K/V block (fewer K/V reads, two
     // softmax warpgroups in flight); one per CTA when two would leave SMs idle.
@@ -416,10 +436,13 @@ int checked_run(cudaStream_t stream, Go go) {
 }
 
 int forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
-                    int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags) {
-    int rc = check_args(q, k, v, out, B, N, H, D, scale, dtype);
+                    int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags,
+                    int64_t Hkv = 0) {
+    int rc = Hkv ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
+                 : check_args(q, k, v, out, B, N, H, D, scale, dtype);
     if (rc) return rc;
-    return checked_run(stream, [&] { return launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags); });
+    return checked_run(stream,
+                       [&] { return launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags, Hkv); });
 }
 
 int forward_varlen_checked(const void* q, const void* k, const void* v, void* out, const int32_t* cu,
@@ -458,6 +481,32 @@ VITATTN_API int vitattn_test_forward_flags(const void* q, const void* k, const v
                                vitattn_stream_t stream, int flags) {
     return forward_checked(q, k, v, out, B, N, H, D, scale, dtype,
                            reinterpret_cast<cudaStream_t>(stream), flags);
+}
+
+int vitattn_forward_gqa(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N, int64_t H,
+                        int64_t Hkv, int64_t D, float scale, int dtype, vitattn_stream_t stream) {
+    return launch(q, k, v, out, B, N, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), 0, Hkv);
+}
+
+int vitattn_forward_gqa_checked(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
+                                int64_t H, int64_t Hkv, int64_t D, float scale, int dtype,
+                                vitattn_stream_t stream) {
+    return forward_checked(q, k, v, out, B, N, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), 0,
+                           Hkv);
+}
+
+// Test hook, deliberately absent from the public header: the checked
+// grouped-query entry with the test flags of vitattn_test_forward_flags.
+VITATTN_API int vitattn_test_forward_gqa_flags(const void* q, const void* k, const void* v, void* out, int64_t B,
+                                               int64_t N, int64_t H, int64_t Hkv, int64_t D, float scale,
+                                               int dtype, vitattn_stream_t stream, int flags) {
+    return forward_checked(q, k, v, out, B, N, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), flags,
+                           Hkv);
+}
+
+int vitattn_check_args_gqa(const void* q, const void* k, const void* v, const void* out, int64_t B, int64_t N,
+                           int64_t H, int64_t Hkv, int64_t D, float scale, int dtype) {
+    return check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype);
 }
 
 int vitattn_forward_varlen(const void* q, const void* k, const void* v, void* out,

@@ -15,6 +15,9 @@ Workloads (token-major ``[B, N, H, D]`` as they leave a ViT's QKV linear):
 - ``doc_page``   1 x 912 x 16 x 80, bf16, Q,K iid N(0, 1.5^2), V iid N(0,1)
   (the 912-patch page of inferencelayer ``vision_gpu.rs``, module doc)
 - ``batched``    32 x 1024 x 16 x 64, bf16, iid N(0,1)
+- ``batched_gqa`` 32 x 1024 x 16 x 64, bf16, iid N(0,1), with 4 key/value heads
+  (k, v are 32 x 1024 x 4 x 64): query head h uses kv head h // 4, the
+  grouped-query ratio of the Gemma-4V vision tower on the hf2q page
 - ``high_res``   2 x 16384 x 16 x 128, bf16, Q = Zq + a*Uq*W, K = Zk + a*Uk*W
   with Z iid N(0,1), U: N x 8 iid N(0,1) per tensor and per (b, h), W: 8 x D
   with orthonormal rows per (b, h) shared by Q and K, and a = sqrt(sqrt(241)-1)
@@ -62,6 +65,7 @@ class Workload:
     qk_std: float = 1.0
     rank8_logit_std: float = 0.0  # 0: iid; >0: shared rank-8 component reaching this logit std
     index: int = 0
+    Hkv: int = 0  # key/value heads (grouped-query attention); 0: as many as query heads
 
     @property
     def scale(self) -> float:
@@ -77,9 +81,13 @@ class Workload:
         return 4.0 * self.B * self.H * self.N * self.N * self.D
 
     @property
+    def kv_heads(self) -> int:
+        return self.Hkv or self.H
+
+    @property
     def io_bytes(self) -> int:
         """Q, K, V read once and O written once, 2 bytes per element."""
-        return 4 * self.B * self.N * self.H * self.D * 2
+        return (2 * self.H + 2 * self.kv_heads) * self.B * self.N * self.D * 2
 
     @property
     def numel(self) -> int:
@@ -94,6 +102,9 @@ WORKLOADS = {
         Workload("doc_page", 1, 912, 16, 80, BF16, qk_std=1.5, index=2),
         Workload("batched", 32, 1024, 16, 64, BF16, index=3),
         Workload("high_res", 2, 16384, 16, 128, BF16, rank8_logit_std=4.0, index=4),
+        # the batched shape with 4 query heads per key/value head (the GQA ratio of the
+        # Gemma-4V vision tower on the hf2q page)
+        Workload("batched_gqa", 32, 1024, 16, 64, BF16, index=7, Hkv=4),
     )
 }
 
@@ -274,6 +285,12 @@ def make_qkv(w: Workload, seed: int | None = None):
     """(q, k, v) uint16 bit arrays of shape [B, N, H, D] for workload ``w``."""
     rng = np.random.Generator(np.random.PCG64(w.seed if seed is None else seed))
     shape = (w.B, w.N, w.H, w.D)
+    if w.Hkv:
+        kv_shape = (w.B, w.N, w.Hkv, w.D)
+        q = rng.standard_normal(size=shape, dtype=np.float32) * np.float32(w.qk_std)
+        k = rng.standard_normal(size=kv_shape, dtype=np.float32) * np.float32(w.qk_std)
+        v = rng.standard_normal(size=kv_shape, dtype=np.float32)
+        return tuple(round_to_bits(x, w.dtype) for x in (q, k, v))
 
     def normal(std: float = 1.0) -> np.ndarray:
         x = rng.standard_normal(size=shape, dtype=np.float32)

@@ -62,6 +62,11 @@ def lib() -> ctypes.CDLL:
         L.vitattn_forward_varlen_checked.argtypes = var
         L.vitattn_test_forward_varlen_flags.argtypes = var + [i32]
         L.vitattn_check_args_varlen.argtypes = var[:-1]
+        gqa = [p, p, p, p, i64, i64, i64, i64, i64, f32, i32, p]
+        L.vitattn_forward_gqa.argtypes = gqa
+        L.vitattn_forward_gqa_checked.argtypes = gqa
+        L.vitattn_test_forward_gqa_flags.argtypes = gqa + [i32]
+        L.vitattn_check_args_gqa.argtypes = gqa[:-1]
         rope = [p, p, p, p, p, p, i64, i64, i64, i32]
         L.vitattn_qkv_rope.argtypes = rope + [p]
         L.vitattn_check_args_qkv_rope.argtypes = rope
@@ -71,7 +76,9 @@ def lib() -> ctypes.CDLL:
                   L.vitattn_forward_host, L.vitattn_check_args, L.vitattn_last_cuda_error,
                   L.vitattn_version, L.vitattn_launches_per_call, L.vitattn_forward_varlen,
                   L.vitattn_forward_varlen_checked, L.vitattn_test_forward_varlen_flags,
-                  L.vitattn_check_args_varlen, L.vitattn_qkv_rope, L.vitattn_check_args_qkv_rope):
+                  L.vitattn_check_args_varlen, L.vitattn_qkv_rope, L.vitattn_check_args_qkv_rope,
+                  L.vitattn_forward_gqa, L.vitattn_forward_gqa_checked, L.vitattn_test_forward_gqa_flags,
+                  L.vitattn_check_args_gqa):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -277,3 +284,54 @@ def qkv_rope(qkv, cos, sin, stream=None):
     if rc != 0:
         raise VitAttnError(rc, "vitattn_qkv_rope")
     return q, k, v
+
+
+def check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype) -> int:
+    """Status the grouped-query argument checks give (pointers as ints); no CUDA call."""
+    return int(lib().vitattn_check_args_gqa(q, k, v, out, B, N, H, Hkv, D, float(scale), dtype))
+
+
+def forward_gqa_ptr(q, k, v, out, B, N, H, Hkv, D, scale, dtype, stream=0, checked=False, flags=0) -> int:
+    """Raw grouped-query call on device pointers (ints); returns the status."""
+    L = lib()
+    args = (q, k, v, out, B, N, H, Hkv, D, float(scale), dtype, stream)
+    if flags:
+        return int(L.vitattn_test_forward_gqa_flags(*args, int(flags)))
+    if checked:
+        return int(L.vitattn_forward_gqa_checked(*args))
+    return int(L.vitattn_forward_gqa(*args))
+
+
+def forward_gqa(q, k, v, out=None, scale=None, stream=None, checked=False):
+    """Grouped-query attention on CUDA tensors: q ``[B, N, H, D]``, k and v
+    ``[B, N, Hkv, D]`` with H a multiple of Hkv; query head h uses key/value
+    head h // (H // Hkv).  ``scale`` defaults to 1/sqrt(D).  Returns ``out``
+    ``[B, N, H, D]``."""
+    import torch
+
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape or k.shape[:2] != q.shape[:2] or k.shape[3] != q.shape[3]:
+        raise ValueError("q must be [B, N, H, D] and k, v [B, N, Hkv, D]")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous")
+    dtype = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    Hkv = k.shape[2]
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor like q")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    with torch.cuda.device(q.device):
+        rc = forward_gqa_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, Hkv, D, scale,
+                             dtype, handle, checked=checked)
+    if rc != 0:
+        raise VitAttnError(rc, "vitattn_forward_gqa")
+    return out
