@@ -115,6 +115,40 @@ def probs(q, k, scale: float, dtype: int, b: int, h: int) -> np.ndarray:
     return P
 
 
+def attention_ext(q, k, v, scale: float, dtype: int, causal: bool = False):
+    """Attention with separate query and key lengths, an optional aligned
+    causal mask, and the log-sum-exp of each row (hanzo-ml
+    ``src/vulkan_backend.rs``, ``flash_attn_gpu``: ``scale`` multiplies
+    Q K^T; ``causal`` lets query ``i`` attend to keys ``j <= i + (Lk - Lq)``).
+
+    ``q``: ``[B, Lq, H, D]``, ``k``, ``v``: ``[B, Lk, H, D]`` (bit patterns of
+    ``dtype``, or float64 with F64).  Returns ``(out [B, Lq, H, D],
+    lse [B, H, Lq])`` in float64, ``lse = log(sum_j exp(scale * q_i . k_j))``
+    over the keys the row sees.  A row that sees no key (only possible when
+    Lq > Lk) gets ``out = 0`` and ``lse = -inf``.  Plain numpy, one (b, h) at
+    a time: the definition written out."""
+    qf, kf, vf = ((x.astype(np.float64) if dtype == F64 else widen(np.ascontiguousarray(x), dtype)) for x in (q, k, v))
+    B, Lq, H, D = qf.shape
+    Lk = kf.shape[1]
+    out = np.zeros((B, Lq, H, D))
+    lse = np.full((B, H, Lq), -np.inf)
+    i = np.arange(Lq)[:, None]
+    j = np.arange(Lk)[None, :]
+    seen = (j <= i + (Lk - Lq)) if causal else np.ones((Lq, Lk), bool)
+    rows = seen.any(axis=1)
+    for b in range(B):
+        for h in range(H):
+            s = scale * (qf[b, :, h] @ kf[b, :, h].T)
+            s = np.where(seen, s, -np.inf)
+            m = np.where(rows, s.max(axis=1), 0.0)
+            e = np.exp(s - m[:, None])
+            tot = e.sum(axis=1)
+            w = np.divide(e, tot[:, None], out=np.zeros_like(e), where=rows[:, None])
+            out[b, :, h] = w @ vf[b, :, h]
+            lse[b, h] = np.where(rows, m + np.log(np.where(rows, tot, 1.0)), -np.inf)
+    return out, lse
+
+
 def attention_gqa(q, k, v, scale: float, dtype: int, mode: int = MODE_TWO_PASS) -> np.ndarray:
     """Grouped-query attention: ``q`` is ``[B, N, H, D]``, ``k`` and ``v`` are
     ``[B, N, Hkv, D]`` with ``H`` a multiple of ``Hkv``; query head ``h``

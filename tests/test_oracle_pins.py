@@ -461,3 +461,60 @@ def test_gqa_oracle_rejects_bad_head_counts():
     with pytest.raises(ValueError):
         oracle.attention_gqa(q, np.zeros((1, 2, 4, 8), np.uint16), np.zeros((1, 2, 4, 8), np.uint16), 1.0,
                              oracle.BF16)
+
+
+# ---------------------------------------------------------------- cross lengths, aligned causal mask, LSE
+
+def _ext_inputs(B, Lq, Lk, H, D, seed, dtype=synth.BF16):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    q = synth.round_to_bits(rng.standard_normal((B, Lq, H, D), dtype=np.float32), dtype)
+    k = synth.round_to_bits(rng.standard_normal((B, Lk, H, D), dtype=np.float32), dtype)
+    v = synth.round_to_bits(rng.standard_normal((B, Lk, H, D), dtype=np.float32), dtype)
+    return q, k, v
+
+
+def test_ext_without_mask_equals_the_plain_oracle_and_its_probabilities():
+    q, k, v = _ext_inputs(2, 9, 9, 3, 8, 140)
+    out, lse = oracle.attention_ext(q, k, v, 0.4, oracle.BF16)
+    np.testing.assert_allclose(out, oracle.attention(q, k, v, 0.4, oracle.BF16), rtol=0, atol=1e-12)
+    qf, kf = oracle.widen(q, oracle.BF16), oracle.widen(k, oracle.BF16)
+    for b in range(2):
+        for h in range(3):
+            s = 0.4 * qf[b, :, h] @ kf[b, :, h].T
+            # p = exp(s - lse) is the softmax the plain oracle exposes
+            np.testing.assert_allclose(np.exp(s - lse[b, h][:, None]), oracle.probs(q, k, 0.4, oracle.BF16, b, h),
+                                       rtol=0, atol=1e-12)
+
+
+def test_ext_causal_rows_see_the_aligned_prefix():
+    Lq, Lk = 5, 8                                     # offset Lk - Lq = 3
+    q, k, v = _ext_inputs(1, Lq, Lk, 2, 8, 141)
+    out, lse = oracle.attention_ext(q, k, v, 0.3, oracle.BF16, causal=True)
+    for i in range(Lq):
+        n = i + 3 + 1                                 # keys 0 .. i + 3
+        sub_out, sub_lse = oracle.attention_ext(q[:, i:i + 1], k[:, :n], v[:, :n], 0.3, oracle.BF16)
+        np.testing.assert_allclose(out[:, i], sub_out[:, 0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[:, :, i], sub_lse[:, :, 0], rtol=0, atol=1e-12)
+
+
+def test_ext_causal_first_row_is_v0_and_lse_is_its_score():
+    q, k, v = _ext_inputs(1, 6, 6, 1, 8, 142)
+    out, lse = oracle.attention_ext(q, k, v, 0.5, oracle.BF16, causal=True)
+    vf, qf, kf = (oracle.widen(x, oracle.BF16) for x in (v, q, k))
+    assert np.array_equal(out[0, 0, 0], vf[0, 0, 0])
+    assert lse[0, 0, 0] == 0.5 * float(qf[0, 0, 0] @ kf[0, 0, 0])
+
+
+def test_ext_rows_that_see_no_key_are_zero_with_lse_minus_inf():
+    q, k, v = _ext_inputs(1, 7, 4, 2, 8, 143)           # offset -3: rows 0..2 see nothing
+    out, lse = oracle.attention_ext(q, k, v, 0.5, oracle.BF16, causal=True)
+    assert np.all(out[:, :3] == 0.0) and np.all(np.isneginf(lse[:, :, :3]))
+    assert np.all(np.isfinite(lse[:, :, 3:]))
+
+
+def test_ext_lse_is_the_log_of_the_exponential_sum():
+    q, k, v = _ext_inputs(1, 4, 6, 1, 8, 144)
+    _, lse = oracle.attention_ext(q, k, v, 0.25, oracle.BF16)
+    qf, kf = oracle.widen(q, oracle.BF16), oracle.widen(k, oracle.BF16)
+    direct = np.log(np.exp(0.25 * qf[0, :, 0] @ kf[0, :, 0].T).sum(axis=1))
+    np.testing.assert_allclose(lse[0, 0], direct, rtol=0, atol=1e-12)
