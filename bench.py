@@ -173,6 +173,14 @@ def oracle_rows(w, q, k, v, rows):
     """The oracle on sampled output rows; returns the flops those rows cost."""
     import oracle
 
+    if isinstance(w, synth.Workload) and w.causal:
+        # the oracle's causal form on whole (b, h) slices: rows -> their (b, h), each computed once
+        H = w.H
+        bh = sorted({(int(r) // H // w.N, int(r) % H) for r in rows})
+        for b, h in bh:
+            oracle.attention_ext(q[b:b + 1, :, h:h + 1], k[b:b + 1, :, h:h + 1], v[b:b + 1, :, h:h + 1], w.scale,
+                                 w.dtype, causal=True)
+        return 4.0 * w.D * w.N * (w.N + 1) / 2 * len(bh)
     if isinstance(w, synth.Workload) and w.Hkv:
         g = w.H // w.Hkv
         oracle.attention_rows(q, np.repeat(k, g, axis=2), np.repeat(v, g, axis=2), w.scale, w.dtype, rows)
@@ -252,6 +260,8 @@ def shape_config(w):
     cfg = {"B": w.B, "N": w.N, "H": w.H, "D": w.D}
     if w.Hkv:
         cfg["Hkv"] = w.Hkv
+    if w.causal:
+        cfg["causal"] = "aligned (query i sees keys j <= i), with the f32 LSE output; flops count N(N+1)/2 pairs"
     return cfg
 
 
@@ -482,6 +492,8 @@ def main():
     w, q, k, v = load_workload(args.workload)
     ragged = isinstance(w, synth.RaggedWorkload)
     gqa = not ragged and bool(w.Hkv)
+    causal = not ragged and w.causal
+    dlse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda") if causal else None
     tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
     dev = torch.device("cuda", local if world > 1 else 0)
 
@@ -506,6 +518,12 @@ def main():
                                           n_seqs, w.H, w.D, w.scale, w.dtype, sh)
             if rc:
                 raise vitattn.VitAttnError(rc, "vitattn_forward_varlen")
+    elif causal:
+        def step():
+            rc = L.vitattn_forward_ext(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), dlse.data_ptr(),
+                                       w.B, w.N, w.N, w.H, w.D, w.scale, 1, w.dtype, sh)
+            if rc:
+                raise vitattn.VitAttnError(rc, "vitattn_forward_ext")
     elif gqa:
         def step():
             rc = L.vitattn_forward_gqa(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B, w.N,
@@ -527,6 +545,10 @@ def main():
         elif gqa:
             rc = vitattn.forward_gqa_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B, w.N,
                                          w.H, w.Hkv, w.D, w.scale, w.dtype, sh, checked=True)
+        elif causal:
+            rc = vitattn.forward_ext_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(),
+                                         dlse.data_ptr(), w.B, w.N, w.N, w.H, w.D, w.scale, True, w.dtype, sh,
+                                         checked=True)
         else:
             rc = vitattn.forward_ptr(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B,
                                      w.N, w.H, w.D, w.scale, w.dtype, sh, checked=True)
@@ -580,14 +602,20 @@ def main():
     hout_p = torch.empty_like(hq).pin_memory()  # like q
     e2e_steps = max(1, args.e2e_steps)
 
-    if ragged or gqa:
+    if ragged or gqa or causal:
+        hlse_p = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory() if causal else None
+
         def e2e_step():
             for d, h in ((dq, hq_p), (dk, hk_p), (dv, hv_p)):
                 d.copy_(h, non_blocking=True)
             if ragged:
                 vitattn.forward_varlen(dq, dk, dv, w.cu_seqlens, out=dout, scale=w.scale, stream=stream)
-            else:
+            elif gqa:
                 vitattn.forward_gqa(dq, dk, dv, out=dout, scale=w.scale, stream=stream)
+            else:
+                _, lse = vitattn.forward_ext(dq, dk, dv, out=dout, scale=w.scale, causal=True, with_lse=True,
+                                             stream=stream)
+                hlse_p.copy_(lse, non_blocking=True)
             hout_p.copy_(dout, non_blocking=True)
     else:
         def e2e_step():
@@ -665,10 +693,11 @@ def main():
             },
             "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": sum(x.numel() for x in (hq, hk, hv)) * 2,
-                    "d2h_bytes_per_step": hq.numel() * 2,
+                    "d2h_bytes_per_step": hq.numel() * 2 + (w.B * w.H * w.N * 4 if causal else 0),
                     "ms_per_step": e2e_ms / e2e_steps,
                     "entry": ("forward_varlen + stream copies" if ragged else
-                              "forward_gqa + stream copies" if gqa else "vitattn_forward_host")},
+                              "forward_gqa + stream copies" if gqa else
+                              "forward_ext (causal, lse) + stream copies" if causal else "vitattn_forward_host")},
             "gpu_launches": args.steps * vitattn.launches_per_call(),
             "clocks": clocks,
             "cpu_baseline": cpu,

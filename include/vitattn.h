@@ -117,6 +117,37 @@ VITATTN_API int vitattn_forward_checked(const void* q, const void* k, const void
                             vitattn_stream_t stream);
 
 /*
+ * vitattn_forward_ext -- separate query and key lengths, an optional aligned
+ * causal mask, and an optional log-sum-exp output.  Source: hanzo-ml
+ * "src/vulkan_backend.rs", `flash_attn_gpu` (q [BH, Lq, D], k/v [BH, Lk, D];
+ * `scale` multiplies Q K^T; `causal` applies aligned causal masking: query qi
+ * attends to keys <= qi + (Lk - Lq)).
+ *   q, out    [B, Lq, H, D];  k, v  [B, Lk, H, D] (token-major, as
+ *             vitattn_forward); Lq, Lk >= 1.
+ *   lse       NULL, or a 16-byte aligned device pointer to [B, H, Lq] float32
+ *             receiving log(sum_j exp(scale * q_i . k_j)) over the keys row i
+ *             sees (natural log).  The probabilities enter the P.V product
+ *             as f16 (see the layout notes above), so lse is that of the
+ *             rounded weights: within ~1e-3 of the exact value.
+ *   causal    nonzero: the aligned causal mask above.  A row that sees no key
+ *             (only when Lq > Lk) is written as 0 with lse = -inf.
+ * Lq = Lk with causal = 0 and lse = NULL is exactly vitattn_forward.
+ */
+VITATTN_API int vitattn_forward_ext(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B,
+                                    int64_t Lq, int64_t Lk, int64_t H, int64_t D, float scale, int causal,
+                                    int dtype, vitattn_stream_t stream);
+
+/* vitattn_forward_ext, then a stream synchronisation and a read of the kernel's status words. */
+VITATTN_API int vitattn_forward_ext_checked(const void* q, const void* k, const void* v, void* out, float* lse,
+                                            int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D, float scale,
+                                            int causal, int dtype, vitattn_stream_t stream);
+
+/* The argument checks of vitattn_forward_ext alone (no CUDA call). */
+VITATTN_API int vitattn_check_args_ext(const void* q, const void* k, const void* v, const void* out,
+                                       const float* lse, int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D,
+                                       float scale, int dtype);
+
+/*
  * vitattn_forward_gqa -- grouped-query attention: H query heads share Hkv
  * key/value heads, query head h using key/value head h / (H / Hkv).
  * Source: hf2q "src/inference/vision/vit_gpu.rs", doc of `vit_repeat_kv_gpu`

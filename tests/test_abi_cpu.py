@@ -187,3 +187,30 @@ def test_gqa_valid_arguments_pass():
 ])
 def test_gqa_argument_errors(kw, code):
     assert check_gqa(**kw) == code
+
+
+# ---------------------------------------------------------------- cross lengths, causal mask, LSE
+
+def check_ext(**kw):
+    Lq, Lk, H, D = kw.get("Lq", 64), kw.get("Lk", 32), 2, 64
+    qb, kb = Lq * H * D * 2, Lk * H * D * 2
+    a = dict(q=A, out=A + qb, k=A + 2 * qb, v=A + 2 * qb + kb, lse=A + 2 * qb + 2 * kb, B=1, Lq=Lq, Lk=Lk, H=H, D=D,
+             scale=0.125, dtype=vitattn.BF16)
+    a.update(kw)
+    return vitattn.check_args_ext(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Lq"], a["Lk"], a["H"],
+                                  a["D"], a["scale"], a["dtype"])
+
+
+def test_ext_valid_arguments_pass():
+    assert check_ext() == 0
+    assert check_ext(lse=0) == 0
+    assert check_ext(Lq=1, Lk=4096) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(k=0), -1), (dict(Lk=0), -2), (dict(Lq=0), -2), (dict(D=60), -3),
+    (dict(dtype=9), -4), (dict(lse=A + 2 * 64 * 256 + 2 * 32 * 256 + 4), -5), (dict(v=A + 8), -5),
+    (dict(out=A + 2 * 64 * 256 + 16), -6), (dict(lse=A + 64 * 256 + 64), -6), (dict(scale=float("inf")), -9),
+])
+def test_ext_argument_errors(kw, code):
+    assert check_ext(**kw) == code

@@ -203,6 +203,10 @@ struct alignas(64) FwdParams {
     int n_items;        // all work items; a CTA takes items blockIdx.x + k * gridDim.x
     int n_kblocks;      // ceil(N / 128) (dense layout; a ragged batch takes it per segment)
     int kv_group;       // query heads per key/value head (1: multi-head; H / Hkv: grouped-query)
+    int Nk;             // keys per (b, h), dense layout (N unless query and key lengths differ)
+    int causal;         // nonzero: query i sees keys j <= i + causal_off only (aligned causal mask)
+    int causal_off;     // Nk - N
+    float* lse;         // optional [B, H, N] f32: log sum_j exp(scale * q_i . k_j); nullptr: not written
     float scale_log2;
     int flags;
     unsigned long long timeout_ns;
@@ -490,6 +494,12 @@ __device__ __forceinline__ void store_row(uint32_t tO, float inv_l, uint8_t* oro
     }
 }
 
+// Zeros for this thread's output row (a query that sees no key).
+__device__ __forceinline__ void store_zero_row(uint8_t* orow, bool row_ok, int D) {
+    if (!row_ok) return;
+    for (int col = 0; col + 8 <= D; col += 8) ptx::st_global_v4(orow + 2 * col, 0u, 0u, 0u, 0u);
+}
+
 // ---------------------------------------------------------------- the kernel
 
 // kLoop: the CTA loops over work items (grid smaller than the item count);
@@ -529,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     // than items only when every item has the same number of query tiles and
     // key blocks, so T and nkb below hold for all of this CTA's items.
     struct Item {
-        int b, h, q0, nt, tok0, n;
+        int b, h, q0, nt, tok0, n, nk;  // n query rows, nk keys (equal except for cross lengths)
     };
     auto item_of = [&](int i) -> Item {
         Item it;
@@ -549,6 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             it.b = 0;
             it.tok0 = seg.start[lo];
             it.n = seg.len[lo];
+            it.nk = it.n;
         } else {
             qg = i % p.n_qgroups;
             const int bh = i / p.n_qgroups;
@@ -556,6 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             it.b = bh / p.H;
             it.tok0 = 0;
             it.n = p.N;
+            it.nk = p.Nk;
         }
         it.q0 = qg * (p.tiles_per_cta * kTileRows);
         it.nt = (p.tiles_per_cta == 2 && it.q0 + kTileRows < it.n) ? 2 : 1;
@@ -564,7 +576,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const int n_my = kLoop ? (p.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 1;
     const Item first = item_of(blockIdx.x);
     const int T = first.nt;
-    const int nkb = kLoop ? p.n_kblocks : (first.n + kBlockKeys - 1) / kBlockKeys;
+    // key blocks of this CTA's items; with the causal mask, only up to the last
+    // key the item's last query row sees (0 if no row sees any key)
+    int nkb;
+    if (kLoop) {
+        nkb = p.n_kblocks;
+    } else {
+        int keys = first.nk;
+        if (p.causal) keys = max(0, min(keys, min(first.q0 + T * kTileRows, first.n) + p.causal_off));
+        nkb = (keys + kBlockKeys - 1) / kBlockKeys;
+    }
     const uint64_t tmo = p.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -888,13 +909,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
                         for (int i = 0; i < 32; ++i) s[32 * q + i] = __uint_as_float(r[q][i]);
                 }
-                const int valid = min(kBlockKeys, it.n - j * kBlockKeys);
-                const bool partial = valid < kBlockKeys;
+                // keys of this block the row sees: the ragged tail, and with the
+                // causal mask the row's own limit (<= 0: none); "partial" is decided
+                // warp-wide because the exp path holds warp-collective TMEM stores
+                int valid = min(kBlockKeys, it.nk - j * kBlockKeys);
+                if (p.causal) valid = min(valid, row + p.causal_off + 1 - j * kBlockKeys);
+                const bool partial = __any_sync(0xffffffffu, valid < kBlockKeys);
                 const float ext = partial ? (neg ? row_extreme<true, true>(s, valid)
                                                  : row_extreme<true, false>(s, valid))
                                           : (neg ? row_extreme<false, true>(s, valid)
                                                  : row_extreme<false, false>(s, valid));
-                const float m_blk = ext * c2;
+                const float m_blk = valid > 0 ? ext * c2 : -INFINITY;
                 const float m_new = fmaxf(m_used, m_blk);
                 const bool need = (m_new - m_used) > kRescaleThreshold;
                 float alpha = 1.f;
@@ -922,13 +947,18 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(bar(kBarPFull + 2 * t + (g & 1)));
             }
-            if (ok) ok = wait_warp(bar(kBarOFull + t), (uint32_t)k & 1u, abort_flag, tmo, 8);
+            if (ok && nkb > 0) ok = wait_warp(bar(kBarOFull + t), (uint32_t)k & 1u, abort_flag, tmo, 8);
             if (ok) {
                 ptx::tc_fence_after();
                 uint8_t* orow =
                     reinterpret_cast<uint8_t*>(p.out) +
                     ((((size_t)it.b * p.N + (size_t)it.tok0 + (size_t)min(row, it.n - 1)) * p.H + it.h) * p.D) * 2;
-                store_row<DP, kBF16>(tO, 1.f / l, orow, row < it.n, p.D);
+                // a row that saw no key (causal, more queries than keys) is 0
+                if (nkb > 0) store_row<DP, kBF16>(tO, l > 0.f ? 1.f / l : 0.f, orow, row < it.n, p.D);
+                else store_zero_row(orow, row < it.n, p.D);
+                if (p.lse != nullptr && row < it.n)
+                    p.lse[((size_t)it.b * p.H + it.h) * p.N + it.tok0 + row] =
+                        l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
                 // O_t has been read (store_row waits for each load): the next
                 // item's first P.V may overwrite it
                 if (kLoop) {

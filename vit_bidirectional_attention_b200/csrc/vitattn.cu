@@ -70,6 +70,29 @@ int check_args(const void* q, const void* k, const void* v, const void* out, int
     return VITATTN_OK;
 }
 
+// Cross lengths: q, out [B, Lq, H, D]; k, v [B, Lk, H, D]; lse (optional) [B, H, Lq] f32.
+int check_args_ext(const void* q, const void* k, const void* v, const void* out, const float* lse, int64_t B,
+                   int64_t Lq, int64_t Lk, int64_t H, int64_t D, float scale, int dtype) {
+    if (!q || !k || !v || !out) return VITATTN_ERR_NULL;
+    if (Lk < 1) return VITATTN_ERR_DIM;
+    // the query side and every shape limit as for self-attention of length Lq, then the key side
+    int rc = check_args(q, q, q, out, B, Lq, H, D, scale, dtype);
+    if (rc) return rc;
+    rc = check_args(k, k, k, k, B, Lk, H, D, scale, dtype);
+    if (rc && rc != VITATTN_ERR_ALIAS) return rc;  // k "aliasing" itself is the stand-in, not an error
+    if ((reinterpret_cast<uintptr_t>(v) & 15u) || (reinterpret_cast<uintptr_t>(lse) & 15u)) return VITATTN_ERR_ALIGN;
+    const uint64_t q_bytes = (uint64_t)B * (uint64_t)Lq * (uint64_t)H * (uint64_t)D * 2u;
+    const uint64_t kv_bytes = (uint64_t)B * (uint64_t)Lk * (uint64_t)H * (uint64_t)D * 2u;
+    if (overlaps2(out, q_bytes, k, kv_bytes) || overlaps2(out, q_bytes, v, kv_bytes)) return VITATTN_ERR_ALIAS;
+    if (lse) {
+        const uint64_t lse_bytes = (uint64_t)B * (uint64_t)H * (uint64_t)Lq * 4u;
+        if (overlaps2(lse, lse_bytes, out, q_bytes) || overlaps2(lse, lse_bytes, q, q_bytes) ||
+            overlaps2(lse, lse_bytes, k, kv_bytes) || overlaps2(lse, lse_bytes, v, kv_bytes))
+            return VITATTN_ERR_ALIAS;
+    }
+    return VITATTN_OK;
+}
+
 // Grouped-query attention: q, out [B, N, H, D]; k, v [B, N, Hkv, D], H a multiple of Hkv.
 int check_args_gqa(const void* q, const void* k, const void* v, const void* out, int64_t B, int64_t N,
                    int64_t H, int64_t Hkv, int64_t D, float scale, int dtype) {
@@ -270,21 +293,25 @@ int ensure_smem(int dp, int dtype, Mode mode, const void* fn) {
 
 // Tensor maps of q, k, v for every column-chunk width, and the shape fields.
 int fill_common(FwdParams* prm, const void* q, const void* k, const void* v, void* out, int64_t B,
-                int64_t N, int64_t H, int64_t D, float scale, int dtype, int flags, int64_t Hkv = 0) {
+                int64_t N, int64_t H, int64_t D, float scale, int dtype, int flags, int64_t Hkv = 0,
+                int64_t Nk = 0) {
     std::memset(prm, 0, sizeof *prm);
     if (Hkv == 0) Hkv = H;  // multi-head: k and v have the query's head count
+    if (Nk == 0) Nk = N;    // self-attention: as many keys as queries
     const int dp = (int)((D + 15) / 16 * 16);
     const void* src[3] = {q, k, v};
     const int64_t heads[3] = {H, Hkv, Hkv};
+    const int64_t lens[3] = {N, Nk, Nk};
     const int nch = vitattn::chunk_count(dp);
     for (int c = 0; c < nch; ++c) {
         const int w = vitattn::chunk_width(dp, c);
         for (int m = 0; m < 3; ++m) {
             CUtensorMap* map = &prm->maps[m][vitattn::width_class(w)];
-            if (!encode_map(map, src[m], dtype, B, N, heads[m], D, w)) return cuda_fail(cudaErrorInvalidValue);
+            if (!encode_map(map, src[m], dtype, B, lens[m], heads[m], D, w)) return cuda_fail(cudaErrorInvalidValue);
         }
     }
     prm->kv_group = (int)(H / Hkv);
+    prm->Nk = (int)Nk;
     prm->out = out;
     prm->B = (int)B;
     prm->N = (int)N;
@@ -310,19 +337,32 @@ int run_kernel(int dp, int dtype, Mode mode, unsigned grid, FwdParams* prm, Seg*
     return VITATTN_OK;
 }
 
+// Cross-length / causal / LSE extras of the dense launch (all off by default).
+struct Ext {
+    int64_t Nk = 0;       // keys per (b, h); 0: N
+    int causal = 0;       // aligned causal mask
+    float* lse = nullptr; // optional [B, H, N] log-sum-exp output
+};
+
 int launch(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
-           int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags, int64_t Hkv = 0) {
-    int rc = Hkv ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
-                 : check_args(q, k, v, out, B, N, H, D, scale, dtype);
+           int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags, int64_t Hkv = 0,
+           const Ext& ext = Ext()) {
+    int rc = ext.Nk ? check_args_ext(q, k, v, out, ext.lse, B, N, ext.Nk, H, D, scale, dtype)
+             : Hkv  ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
+                    : check_args(q, k, v, out, B, N, H, D, scale, dtype);
     if (rc) return rc;
+    const int64_t Nk = ext.Nk ? ext.Nk : N;
     const int dp = (int)((D + 15) / 16 * 16);
     int num_sms = 0;
     rc = device_info(&num_sms);
     if (rc) return rc;
 
     FwdParams prm;
-    rc = fill_common(&prm, q, k, v, out, B, N, H, D, scale, dtype, flags, Hkv);
+    rc = fill_common(&prm, q, k, v, out, B, N, H, D, scale, dtype, flags, Hkv, Nk);
     if (rc) return rc;
+    prm.causal = ext.causal ? 1 : 0;
+    prm.causal_off = (int)(Nk - N);
+    prm.lse = ext.lse;
     // Two query tiles per CTA share each K/V block (fewer K/V reads, two
     // softmax warpgroups in flight); one per CTA when two would leave SMs idle.
     const uint64_t pairs = (uint64_t)B * (uint64_t)H * (uint64_t)((N + 255) / 256);
@@ -331,14 +371,15 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     if (flags & vitattn::kFlagForceOneTile) prm.tiles_per_cta = 1;
     prm.n_qgroups = (int)((N + 128 * prm.tiles_per_cta - 1) / (128 * prm.tiles_per_cta));
     prm.n_items = (int)((uint64_t)B * (uint64_t)H * (uint64_t)prm.n_qgroups);
-    prm.n_kblocks = (int)((N + 127) / 128);
+    prm.n_kblocks = (int)((Nk + 127) / 128);
 
     // Persistent grid (one CTA per SM, each looping over work items) when there
     // are more items than SMs, the items are short enough (at most 32 key
     // blocks) for the per-CTA start-up and epilogue to matter, and every item
     // has the same number of query tiles (all have two unless the last group
     // of a head is a single tile); otherwise one CTA per item.
-    const bool uniform = prm.tiles_per_cta == 1 || (N % 256 == 0 || N % 256 > 128);
+    // (the causal mask gives items different key-block counts: one CTA per item)
+    const bool uniform = !prm.causal && (prm.tiles_per_cta == 1 || (N % 256 == 0 || N % 256 > 128));
     unsigned grid = (unsigned)prm.n_items;
     if (uniform && prm.n_items > num_sms && prm.n_kblocks <= 32) grid = (unsigned)num_sms;
     if (uniform && (flags & vitattn::kFlagTinyGrid) && grid > 3u) grid = 3u;
@@ -437,12 +478,13 @@ int checked_run(cudaStream_t stream, Go go) {
 
 int forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
                     int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags,
-                    int64_t Hkv = 0) {
-    int rc = Hkv ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
-                 : check_args(q, k, v, out, B, N, H, D, scale, dtype);
+                    int64_t Hkv = 0, const Ext& ext = Ext()) {
+    int rc = ext.Nk ? check_args_ext(q, k, v, out, ext.lse, B, N, ext.Nk, H, D, scale, dtype)
+             : Hkv  ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
+                    : check_args(q, k, v, out, B, N, H, D, scale, dtype);
     if (rc) return rc;
     return checked_run(stream,
-                       [&] { return launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags, Hkv); });
+                       [&] { return launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags, Hkv, ext); });
 }
 
 int forward_varlen_checked(const void* q, const void* k, const void* v, void* out, const int32_t* cu,
@@ -481,6 +523,49 @@ VITATTN_API int vitattn_test_forward_flags(const void* q, const void* k, const v
                                vitattn_stream_t stream, int flags) {
     return forward_checked(q, k, v, out, B, N, H, D, scale, dtype,
                            reinterpret_cast<cudaStream_t>(stream), flags);
+}
+
+int vitattn_forward_ext(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B, int64_t Lq,
+                        int64_t Lk, int64_t H, int64_t D, float scale, int causal, int dtype,
+                        vitattn_stream_t stream) {
+    Ext ext;
+    ext.Nk = Lk < 1 ? -1 : Lk;  // a non-positive Lk is reported by the checks
+    ext.causal = causal;
+    ext.lse = lse;
+    if (Lk < 1) return check_args_ext(q, k, v, out, lse, B, Lq, Lk, H, D, scale, dtype);
+    return launch(q, k, v, out, B, Lq, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), 0, 0, ext);
+}
+
+int vitattn_forward_ext_checked(const void* q, const void* k, const void* v, void* out, float* lse, int64_t B,
+                                int64_t Lq, int64_t Lk, int64_t H, int64_t D, float scale, int causal, int dtype,
+                                vitattn_stream_t stream) {
+    if (Lk < 1) return check_args_ext(q, k, v, out, lse, B, Lq, Lk, H, D, scale, dtype);
+    Ext ext;
+    ext.Nk = Lk;
+    ext.causal = causal;
+    ext.lse = lse;
+    return forward_checked(q, k, v, out, B, Lq, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), 0, 0,
+                           ext);
+}
+
+// Test hook, deliberately absent from the public header: the checked
+// cross-length / causal entry with the test flags of vitattn_test_forward_flags.
+VITATTN_API int vitattn_test_forward_ext_flags(const void* q, const void* k, const void* v, void* out, float* lse,
+                                               int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D,
+                                               float scale, int causal, int dtype, vitattn_stream_t stream,
+                                               int flags) {
+    if (Lk < 1) return check_args_ext(q, k, v, out, lse, B, Lq, Lk, H, D, scale, dtype);
+    Ext ext;
+    ext.Nk = Lk;
+    ext.causal = causal;
+    ext.lse = lse;
+    return forward_checked(q, k, v, out, B, Lq, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), flags,
+                           0, ext);
+}
+
+int vitattn_check_args_ext(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                           int64_t B, int64_t Lq, int64_t Lk, int64_t H, int64_t D, float scale, int dtype) {
+    return check_args_ext(q, k, v, out, lse, B, Lq, Lk, H, D, scale, dtype);
 }
 
 int vitattn_forward_gqa(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N, int64_t H,

@@ -18,6 +18,9 @@ Workloads (token-major ``[B, N, H, D]`` as they leave a ViT's QKV linear):
 - ``batched_gqa`` 32 x 1024 x 16 x 64, bf16, iid N(0,1), with 4 key/value heads
   (k, v are 32 x 1024 x 4 x 64): query head h uses kv head h // 4, the
   grouped-query ratio of the Gemma-4V vision tower on the hf2q page
+- ``batched_causal`` 32 x 1024 x 16 x 64, bf16, iid N(0,1), with the aligned causal
+  mask (query i sees keys j <= i) and the log-sum-exp output; flops count the
+  N(N+1)/2 admitted query-key pairs
 - ``high_res``   2 x 16384 x 16 x 128, bf16, Q = Zq + a*Uq*W, K = Zk + a*Uk*W
   with Z iid N(0,1), U: N x 8 iid N(0,1) per tensor and per (b, h), W: 8 x D
   with orthonormal rows per (b, h) shared by Q and K, and a = sqrt(sqrt(241)-1)
@@ -66,6 +69,7 @@ class Workload:
     rank8_logit_std: float = 0.0  # 0: iid; >0: shared rank-8 component reaching this logit std
     index: int = 0
     Hkv: int = 0  # key/value heads (grouped-query attention); 0: as many as query heads
+    causal: bool = False  # aligned causal mask (query i sees keys j <= i), with the LSE output
 
     @property
     def scale(self) -> float:
@@ -77,8 +81,10 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """4*B*H*N^2*D: the two contractions QK^T and PV, two flops per MAC."""
-        return 4.0 * self.B * self.H * self.N * self.N * self.D
+        """4*B*H*N^2*D: the two contractions QK^T and PV, two flops per MAC
+        (with the causal mask only the N(N+1)/2 query-key pairs it admits)."""
+        pairs = self.N * (self.N + 1) / 2 if self.causal else self.N * self.N
+        return 4.0 * self.B * self.H * pairs * self.D
 
     @property
     def kv_heads(self) -> int:
@@ -105,6 +111,8 @@ WORKLOADS = {
         # the batched shape with 4 query heads per key/value head (the GQA ratio of the
         # Gemma-4V vision tower on the hf2q page)
         Workload("batched_gqa", 32, 1024, 16, 64, BF16, index=7, Hkv=4),
+        # the batched shape with the aligned causal mask and the LSE output
+        Workload("batched_causal", 32, 1024, 16, 64, BF16, index=8, causal=True),
     )
 }
 

@@ -62,6 +62,11 @@ def lib() -> ctypes.CDLL:
         L.vitattn_forward_varlen_checked.argtypes = var
         L.vitattn_test_forward_varlen_flags.argtypes = var + [i32]
         L.vitattn_check_args_varlen.argtypes = var[:-1]
+        ext = [p, p, p, p, p, i64, i64, i64, i64, i64, f32, i32, i32, p]
+        L.vitattn_forward_ext.argtypes = ext
+        L.vitattn_forward_ext_checked.argtypes = ext
+        L.vitattn_test_forward_ext_flags.argtypes = ext + [i32]
+        L.vitattn_check_args_ext.argtypes = [p, p, p, p, p, i64, i64, i64, i64, i64, f32, i32]
         gqa = [p, p, p, p, i64, i64, i64, i64, i64, f32, i32, p]
         L.vitattn_forward_gqa.argtypes = gqa
         L.vitattn_forward_gqa_checked.argtypes = gqa
@@ -78,7 +83,8 @@ def lib() -> ctypes.CDLL:
                   L.vitattn_forward_varlen_checked, L.vitattn_test_forward_varlen_flags,
                   L.vitattn_check_args_varlen, L.vitattn_qkv_rope, L.vitattn_check_args_qkv_rope,
                   L.vitattn_forward_gqa, L.vitattn_forward_gqa_checked, L.vitattn_test_forward_gqa_flags,
-                  L.vitattn_check_args_gqa):
+                  L.vitattn_check_args_gqa, L.vitattn_forward_ext, L.vitattn_forward_ext_checked,
+                  L.vitattn_test_forward_ext_flags, L.vitattn_check_args_ext):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -335,3 +341,58 @@ def forward_gqa(q, k, v, out=None, scale=None, stream=None, checked=False):
     if rc != 0:
         raise VitAttnError(rc, "vitattn_forward_gqa")
     return out
+
+
+def check_args_ext(q, k, v, out, lse, B, Lq, Lk, H, D, scale, dtype) -> int:
+    """Status the cross-length / causal argument checks give (pointers as ints); no CUDA call."""
+    return int(lib().vitattn_check_args_ext(q, k, v, out, lse, B, Lq, Lk, H, D, float(scale), dtype))
+
+
+def forward_ext_ptr(q, k, v, out, lse, B, Lq, Lk, H, D, scale, causal, dtype, stream=0, checked=False,
+                    flags=0) -> int:
+    """Raw cross-length / causal / LSE call on device pointers (ints; lse may be 0)."""
+    L = lib()
+    args = (q, k, v, out, lse or None, B, Lq, Lk, H, D, float(scale), int(bool(causal)), dtype, stream)
+    if flags:
+        return int(L.vitattn_test_forward_ext_flags(*args, int(flags)))
+    if checked:
+        return int(L.vitattn_forward_ext_checked(*args))
+    return int(L.vitattn_forward_ext(*args))
+
+
+def forward_ext(q, k, v, out=None, scale=None, causal=False, with_lse=False, stream=None, checked=False):
+    """Attention with query length Lq and key length Lk on CUDA tensors: q
+    ``[B, Lq, H, D]``, k and v ``[B, Lk, H, D]``; ``causal`` lets query i see
+    keys j <= i + (Lk - Lq) only.  Returns ``out`` ``[B, Lq, H, D]``, or
+    ``(out, lse)`` with ``lse`` float32 ``[B, H, Lq]`` when ``with_lse``."""
+    import torch
+
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape or (k.shape[0], k.shape[2], k.shape[3]) != (
+            q.shape[0], q.shape[2], q.shape[3]):
+        raise ValueError("q must be [B, Lq, H, D] and k, v [B, Lk, H, D]")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k, v must be contiguous")
+    dtype = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    B, Lq, H, D = q.shape
+    Lk = k.shape[1]
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor like q")
+    lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device) if with_lse else None
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    with torch.cuda.device(q.device):
+        rc = forward_ext_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr() if lse is not None else 0, B, Lq, Lk, H, D, scale, causal, dtype,
+                             handle, checked=checked)
+    if rc != 0:
+        raise VitAttnError(rc, "vitattn_forward_ext")
+    return (out, lse) if with_lse else out
