@@ -54,7 +54,8 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAK_TFLOPS = 1590.0  # the pool's earlier measurement, used only without MEASURED_PEAKS.json
 DATASHEET_PEAK_TFLOPS = 2250.0
 KERNEL_SOURCES = ["vit_bidirectional_attention_b200/csrc/fwd_kernel.cuh",
-                  "vit_bidirectional_attention_b200/csrc/ptx.cuh"]
+                  "vit_bidirectional_attention_b200/csrc/ptx.cuh",
+                  "vit_bidirectional_attention_b200/csrc/rope_kernel.cuh"]
 
 
 def parse():
