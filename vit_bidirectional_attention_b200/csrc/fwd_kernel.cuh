@@ -562,6 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             it.nk = it.n;
         } else {
             qg = i % p.n_qgroups;
+            // with the causal mask a later query group sees more keys: take each
+            // head's longest group first, so the grid's last CTAs are short ones
+            if (p.causal) qg = p.n_qgroups - 1 - qg;
             const int bh = i / p.n_qgroups;
             it.h = bh % p.H;
             it.b = bh / p.H;
