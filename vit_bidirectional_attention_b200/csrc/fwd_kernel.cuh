@@ -82,7 +82,7 @@ namespace vitattn {
 constexpr int kTileRows = 128;    // query rows per tile = TMEM lanes
 constexpr int kBlockKeys = 128;   // keys per K/V block
 constexpr int kTilesPerCta = 2;
-constexpr int kStages = 4;        // K/V ring slots (K_j, V_j, K_j+1, V_j+1)
+constexpr int kMaxStages = 4;     // K/V ring slots (K_j, V_j, K_j+1, V_j+1)
 constexpr int kThreads = 384;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -102,10 +102,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when the max g
 constexpr int kMaxQBufs = 2;
 constexpr int kBarQFull = 0;                         // [kMaxQBufs][2 tiles] Q loaded
 constexpr int kBarQEmpty = kBarQFull + 2 * kMaxQBufs; // [kMaxQBufs][2 tiles] last S read it
-constexpr int kBarKvFull = kBarQEmpty + 2 * kMaxQBufs;  // [kStages]
-constexpr int kBarKvEmpty = kBarKvFull + kStages;    // [kStages]
+constexpr int kBarKvFull = kBarQEmpty + 2 * kMaxQBufs;  // [kMaxStages]
+constexpr int kBarKvEmpty = kBarKvFull + kMaxStages; // [kMaxStages]
 constexpr int kMaxSBufs = 3;
-constexpr int kBarSFull = kBarKvEmpty + kStages;     // [kMaxSBufs] one per S buffer
+constexpr int kBarSFull = kBarKvEmpty + kMaxStages;  // [kMaxSBufs] one per S buffer
 // [2 tiles][2] P written (and O rescaled) for blocks of even / odd index: with
 // the S look-ahead a tile's softmax can finish block j+1 before the MMA warp
 // has consumed block j, and one barrier per tile could then run two phases
@@ -114,8 +114,8 @@ constexpr int kBarPFull = kBarSFull + kMaxSBufs;
 constexpr int kBarOReady = kBarPFull + 4;            // [2] per tile: a P.V product finished
 constexpr int kBarOFull = kBarOReady + 2;            // [2] per tile: the item's last P.V finished
 constexpr int kBarOEmpty = kBarOFull + 2;            // [2] per tile: the epilogue has read O
-constexpr int kBarVReady = kBarOEmpty + 2;           // [2] bf16: V block of even / odd index is f16
-constexpr int kBarDrain = kBarVReady + 2;            // [1]
+constexpr int kBarVReady = kBarOEmpty + 2;           // [kMaxStages / 2] bf16: the V slot's block is f16
+constexpr int kBarDrain = kBarVReady + kMaxStages / 2;  // [1]
 constexpr int kNumBars = kBarDrain + 1;
 
 // Status codes written to g_vitattn_status (0 = fine).
@@ -171,8 +171,11 @@ __host__ __device__ constexpr bool pv_done_needed(int ns, int ntiles) { return n
 // one runs) when a CTA loops over items and that fits in shared memory, i.e.
 // up to DP = 112.
 __host__ __device__ constexpr int q_buffers(int dp, bool loop) { return (loop && dp <= 112) ? 2 : 1; }
+// K/V ring slots for a padded head dim (even: K in even slots, V in odd ones).
+__host__ __device__ constexpr int kv_stages(int dp) { return kMaxStages; }
+static_assert(kMaxStages % 2 == 0, "K and V alternate in the ring");
 __host__ __device__ constexpr int smem_bytes(int dp, bool loop) {
-    return (q_buffers(dp, loop) * kTilesPerCta + kStages) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
+    return (q_buffers(dp, loop) * kTilesPerCta + kv_stages(dp)) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
 }
 
 // Ragged batches (several images' tokens packed along one axis, start
@@ -516,6 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     static_assert(!(kLoop && kVarlen), "ragged batches run one work item per CTA");
 
     constexpr int NQ = q_buffers(DP, kLoop);
+    constexpr int kStages = kv_stages(DP);
+    constexpr int kVSlots = kStages / 2;  // V_g sits in V slot g % kVSlots, its use g / kVSlots
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -596,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             ptx::mbar_init(bar(kBarQFull + i), 1);
             ptx::mbar_init(bar(kBarQEmpty + i), 1);
         }
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kMaxStages; ++s) {
             ptx::mbar_init(bar(kBarKvFull + s), 1);
             ptx::mbar_init(bar(kBarKvEmpty + s), 1);
         }
@@ -607,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             ptx::mbar_init(bar(kBarOReady + t), 1);
             ptx::mbar_init(bar(kBarOFull + t), 1);
             ptx::mbar_init(bar(kBarOEmpty + t), 4 * 32);
-            ptx::mbar_init(bar(kBarVReady + t), 2 * 32);
+            for (int vs = t; vs < kMaxStages / 2; vs += 2) ptx::mbar_init(bar(kBarVReady + vs), 2 * 32);
         }
         ptx::mbar_init(bar(kBarDrain), 1);
         *abort_flag = 0;
@@ -797,13 +802,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 return true;
             };
             // O_t += P V_j; V_j is waited for by its first unit (landed, and for
-            // bf16 inputs converted to f16) and released after its last.  The
-            // converter is at most two blocks ahead (it needs V_j+2's slot, which
-            // the last P.V of block j frees), so the parity of V-ready is unambiguous.
+            // bf16 inputs converted to f16) and released after its last.  V-ready
+            // is per V slot: the converter reaches the slot's next block only after
+            // it lands there, which needs the last P.V of this one, so the parity is
+            // unambiguous.
             auto issue_pv = [&](const Cursor& c) -> bool {
                 const int t = c.t, j = c.j, g = c.g;
                 if (t == 0 &&
-                    !(kBF16 ? wait_warp(bar(kBarVReady + (g & 1)), (uint32_t)(g >> 1) & 1u, abort_flag, tmo, 4)
+                    !(kBF16 ? wait_warp(bar(kBarVReady + g % kVSlots), (uint32_t)(g / kVSlots) & 1u, abort_flag,
+                                        tmo, 4)
                             : wait_warp(bar(kBarKvFull + kv_slot(2 * g + 1)), kv_parity(2 * g + 1), abort_flag,
                                        tmo, 4)))
                     return false;
@@ -860,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 break;
             vmax = convert_v_tile<TILE>(base_ptr + (sKV - base) + slot * TILE, ct, vmax);
             ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(bar(kBarVReady + (g & 1)));
+            ptx::mbar_arrive(bar(kBarVReady + g % kVSlots));
         }
         if (vmax >= 65536.f) atomicOr(&g_vitattn_range, 1u);
     }
