@@ -18,7 +18,7 @@ from vit_bidirectional_attention_b200 import synth, vitattn
 
 pytestmark = pytest.mark.gpu
 
-FORCE_TWO_TILES, FORCE_ONE_TILE = 2, 4
+FORCE_TWO_TILES, FORCE_ONE_TILE, TINY_GRID = 2, 4, 8
 
 
 def to_dev(bits, dtype):
@@ -106,3 +106,24 @@ def test_python_entry_returns_out_and_lse(cuda_device):
     out, lse = vitattn.forward_ext(tq, tk, tv, causal=True, with_lse=True, checked=True)
     ref, lse_ref = oracle.attention_ext(q, k, v, 1.0 / math.sqrt(72), synth.F16, causal=True)
     check(from_dev(out, synth.F16), ref, lse.cpu().numpy().astype(np.float64), lse_ref, "python entry")
+
+
+@pytest.mark.parametrize("flags", [FORCE_TWO_TILES | TINY_GRID, FORCE_ONE_TILE | TINY_GRID])
+@pytest.mark.parametrize("Lq,Lk", [(512, 512), (256, 640), (384, 384)])
+def test_causal_many_heads_and_groups(cuda_device, Lq, Lk, flags):
+    """Causal launches with several heads and query groups per head (work
+    items of different key-block counts, each head's longest group first);
+    the tiny-grid flag must not change anything for them."""
+    q, k, v = inputs(3, Lq, Lk, 3, 64, synth.BF16, seed=9900 + Lq + Lk + flags)
+    got, lse = run_ext(q, k, v, 0.125, True, synth.BF16, flags)
+    ref, lse_ref = oracle.attention_ext(q, k, v, 0.125, synth.BF16, causal=True)
+    check(got, ref, lse, lse_ref, f"Lq={Lq} Lk={Lk} flags={flags}")
+
+
+def test_causal_launch_with_more_items_than_sms(cuda_device):
+    """4 x 1024 x 16 x 64: 256 work items of 2 to 8 key blocks, more than the
+    SMs (one CTA per item)."""
+    q, k, v = inputs(4, 1024, 1024, 16, 64, synth.BF16, seed=9950)
+    got, lse = run_ext(q, k, v, 0.125, True, synth.BF16)
+    ref, lse_ref = oracle.attention_ext(q, k, v, 0.125, synth.BF16, causal=True)
+    check(got, ref, lse, lse_ref, "causal 4x1024x16x64")
