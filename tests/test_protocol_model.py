@@ -1,0 +1,48 @@
+"""The attention kernel's barrier protocol, replayed on the CPU under random
+schedules (``tests/protocol_model.py``): every configuration the kernel can
+launch -- one or two query tiles, two or three S buffers, one or two Q
+buffers, CTAs looping over items or not, bf16 (with the V converter) or f16 --
+must never let a parity wait pass on the wrong phase and never deadlock."""
+import itertools
+
+import pytest
+
+from protocol_model import run
+
+CONFIGS = [
+    (T, NS, NQ, loop, bf16)
+    for T, NS, NQ, loop, bf16 in itertools.product([1, 2], [2, 3], [1, 2], [False, True], [False, True])
+    if loop or NQ == 1
+]
+
+
+@pytest.mark.parametrize("T,NS,NQ,loop,bf16", CONFIGS)
+def test_protocol_has_no_aliasing_or_deadlock(T, NS, NQ, loop, bf16):
+    for nkb in (1, 2, 3, 5, 8):
+        for n_my in ((1, 2, 3) if loop else (1,)):
+            for seed in range(12):
+                run(T, NS, NQ, nkb, n_my, loop, bf16, seed)
+
+
+def test_the_model_catches_a_planted_mistake():
+    """Sanity of the checker itself: with a single "P written" barrier per
+    tile instead of one per block parity, some schedule lets a softmax run two
+    phases ahead of the MMA warp, and the model reports the aliased wait."""
+    import inspect
+    import types
+
+    import protocol_model
+
+    text = inspect.getsource(protocol_model)
+    mutant = text.replace('("wait", ("p_full", t, g & 1), g >> 1)', '("wait", ("p_full", t, 0), g)').replace(
+        '("arrive", ("p_full", t, g & 1), 128)', '("arrive", ("p_full", t, 0), 128)')
+    assert mutant != text
+    mod = types.ModuleType("protocol_model_mutant")
+    exec(compile(mutant, "protocol_model_mutant", "exec"), mod.__dict__)
+    failures = 0
+    for seed in range(200):
+        try:
+            mod.run(2, 3, 1, 8, 1, False, True, seed)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
