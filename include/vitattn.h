@@ -18,10 +18,21 @@
  * "src/vulkan_backend.rs", `flash_attn_gpu` (the (q, k, v, sizes, scale)
  * calling shape and argument checks before dispatch).
  *
+ * Entry points (each documented below):
+ *   vitattn_forward          the operation above (self-attention, Lq = Lk = N)
+ *   vitattn_forward_varlen   a ragged batch of images packed along one axis
+ *   vitattn_forward_gqa      grouped-query attention (fewer key/value heads)
+ *   vitattn_forward_ext      Lq != Lk, aligned causal mask, log-sum-exp output
+ *   vitattn_qkv_rope         the prologue: packed QKV split + rotary embedding
+ *   vitattn_forward_host     vitattn_forward from host buffers (copies enqueued)
+ *   ..._checked, ..._check_args*, vitattn_strerror, vitattn_last_cuda_error,
+ *   vitattn_version, vitattn_launches_per_call: synchronising variants for
+ *   tests, argument checks alone, status text, versioning.
+ *
  * Layout.  q, k, v and out are dense, token-major [B, N, H, D] tensors with D
  * contiguous: element (b, i, h, d) at ((b*N + i)*H + h)*D + d.  That is the
  * layout a QKV linear produces once its output is split into three.
- * Lq = Lk = N (self-attention).  out has the dtype of the inputs; products
+ * Lq = Lk = N (self-attention) for vitattn_forward.  out has the dtype of the inputs; products
  * and sums accumulate in fp32.  The probabilities enter the P.V product as
  * f16 for both dtypes (f16 carries three more mantissa bits than bf16), and
  * for bf16 inputs V is converted to f16 for that product: exact for
@@ -35,7 +46,7 @@
  * frees caller memory.  out must not overlap q, k or v.
  *
  * Streams and errors.  Calls enqueue work on `stream` and return without
- * synchronising (except vitattn_forward_checked).  Every argument is checked
+ * synchronising (except the ..._checked entries).  Every argument is checked
  * before anything is enqueued; a failed check returns a negative status and
  * enqueues nothing.  A CUDA error raised while enqueueing returns
  * VITATTN_ERR_CUDA (its cudaError_t value via vitattn_last_cuda_error()).
