@@ -32,8 +32,8 @@
  * Layout.  q, k, v and out are dense, token-major [B, N, H, D] tensors with D
  * contiguous: element (b, i, h, d) at ((b*N + i)*H + h)*D + d.  That is the
  * layout a QKV linear produces once its output is split into three.
- * Lq = Lk = N (self-attention) for vitattn_forward.  out has the dtype of the inputs; products
- * and sums accumulate in fp32.  The probabilities enter the P.V product as
+ * Lq = Lk = N (self-attention) for vitattn_forward.  out has the dtype of the
+ * inputs; products and sums accumulate in fp32.  The probabilities enter the P.V product as
  * f16 for both dtypes (f16 carries three more mantissa bits than bf16), and
  * for bf16 inputs V is converted to f16 for that product: exact for
  * |v| < 65536 outside f16's subnormal range (|v| < 2^-14, where the absolute
