@@ -3,9 +3,12 @@
 Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product path (the CUDA library and
 its Python binding) never imports it, and it imports nothing from them: the
-two share no code.  The arithmetic lives in ``attention_oracle.c`` (plain C,
-double precision, OpenMP over rows); this module only compiles it with gcc and
-marshals numpy arrays through ctypes.
+two share no code.  The attention arithmetic lives in ``attention_oracle.c``
+(plain C, double precision, OpenMP over rows); this module compiles it with
+gcc and marshals numpy arrays through ctypes.  The ragged and grouped-query
+forms call the same C routine (per image, or on replicated key/value heads);
+the cross-length / causal form and the prologue functions (``qkv_rope``,
+``qkv_norm_rope``) are plain numpy in float64.
 
 What it computes, per batch b and head h, on token-major ``[B, N, H, D]``
 inputs (hf2q ``src/inference/vision/vit_gpu.rs``, doc of ``vit_attention_gpu``
@@ -235,6 +238,34 @@ def qkv_rope(qkv, cos, sin, dtype: int):
         return t * c + rot * s
 
     return rope(x[:, 0]), rope(x[:, 1]), x[:, 2].copy()
+
+
+def qkv_norm_rope(qkv, cos, sin, q_norm_w, k_norm_w, eps: float, dtype: int):
+    """The prologue with a per-head RMS norm of q and k ahead of the rotary
+    embedding (inferencelayer ``src/vision_gpu.rs``, ``GLM_QKV_QKNORM_ROPE``
+    and its doc, GLM-OCR vision tower: split the packed qkv; normalise each
+    head's q row and k row over its ``head_dim`` elements by the root of
+    their mean square plus ``eps``, times a per-element weight; only then
+    rotate; v passes through).
+
+    ``qkv``, ``cos``, ``sin``, ``dtype`` as in :func:`qkv_rope`;
+    ``q_norm_w``, ``k_norm_w``: ``[D]`` weights (one vector for all heads);
+    ``eps`` >= 0.  Returns (q, k, v) as float64 ``[T, H, D]``, unrounded::
+
+        y[d]  = x[d] / sqrt(mean_e x[e]^2 + eps) * w[d]
+        x'[d] = y[d] * cos[d] + rotate_half(y)[d] * sin[d]
+    """
+    T, three, H, D = qkv.shape
+    if three != 3:
+        raise ValueError("qkv must be [T, 3, H, D]")
+    x = qkv.astype(np.float64) if dtype == F64 else widen(np.ascontiguousarray(qkv), dtype)
+
+    def rms_norm(t, w):
+        ms = np.mean(t * t, axis=-1, keepdims=True)
+        return t / np.sqrt(ms + float(eps)) * np.asarray(w, np.float64)
+
+    normed = np.stack([rms_norm(x[:, 0], q_norm_w), rms_norm(x[:, 1], k_norm_w), x[:, 2]], axis=1)
+    return qkv_rope(normed, cos, sin, F64)
 
 
 def widen(bits: np.ndarray, dtype: int) -> np.ndarray:

@@ -426,6 +426,90 @@ def test_rope_hand_fixture():
     assert v[0, 0].tolist() == [9.0, 10.0, 11.0, 12.0]
 
 
+# ---------------------------------------------------------------- prologue with q/k RMS norm
+
+def test_norm_rope_unit_weights_give_unit_rms_per_head():
+    """w = 1, eps = 0, identity tables: every output q and k head row has mean
+    square exactly 1 (the mean is over D, not a sum), v is untouched."""
+    qkv, _, _ = _rope_case(5, 3, 24, 130)
+    ones, zeros = np.ones((5, 24), np.float32), np.zeros((5, 24), np.float32)
+    w = np.ones(24)
+    q, k, v = oracle.qkv_norm_rope(qkv, ones, zeros, w, w, 0.0, oracle.BF16)
+    for t in (q, k):
+        np.testing.assert_allclose(np.mean(t * t, axis=-1), 1.0, rtol=0, atol=1e-13)
+    assert np.array_equal(v, oracle.widen(qkv, oracle.BF16)[:, 2])
+
+
+def test_norm_rope_is_scale_invariant_without_eps():
+    qkv, c, s = _rope_case(4, 2, 16, 131)
+    x = oracle.widen(qkv, oracle.BF16)
+    w = rnd((16,), 132)
+    a = oracle.qkv_norm_rope(x, c, s, w, w[::-1], 0.0, oracle.F64)
+    b = oracle.qkv_norm_rope(x * 37.5, c, s, w, w[::-1], 0.0, oracle.F64)
+    for i in (0, 1):
+        np.testing.assert_allclose(b[i], a[i], rtol=1e-13, atol=1e-13)
+
+
+def test_norm_rope_constant_row_with_eps_closed_form():
+    """x = 3 everywhere, eps = 7: mean square 9, 3 / sqrt(9 + 7) = 3/4, so
+    under identity tables q = 0.75 * wq and k = 0.75 * wk (eps inside the
+    root and added to the mean; the two weight vectors kept apart)."""
+    D = 8
+    qkv = np.full((1, 3, 2, D), 3.0)
+    wq = np.arange(1.0, D + 1.0)
+    wk = -np.arange(D, 0.0, -1.0)
+    q, k, v = oracle.qkv_norm_rope(qkv, np.ones((1, D)), np.zeros((1, D)), wq, wk, 7.0, oracle.F64)
+    assert np.array_equal(q, np.broadcast_to(0.75 * wq, q.shape))
+    assert np.array_equal(k, np.broadcast_to(0.75 * wk, k.shape))
+    assert np.array_equal(v, qkv[:, 2])
+
+
+@pytest.mark.parametrize("j", [0, 2, 5, 7])
+def test_norm_rope_one_hot_under_quarter_turn_pins_the_order(j):
+    """x = -2 e_j, cos = 0, sin = 1 (the rotation is rotate_half itself),
+    eps = 0: the norm gives -sqrt(D) e_j * w_j, then rotate_half moves it to
+    j + D/2 (same sign) or j - D/2 (negated).  Rotating first and normalising
+    after would pick up w at the destination instead of w_j."""
+    D, half = 8, 4
+    qkv = np.zeros((1, 3, 1, D))
+    qkv[0, 0, 0, j] = -2.0
+    qkv[0, 1, 0, j] = 5.0
+    wq = np.array([1.5, -2.0, 0.25, 3.0, 0.5, 4.0, -1.0, 2.5])
+    wk = wq[::-1].copy()
+    q, k, _ = oracle.qkv_norm_rope(qkv, np.zeros((1, D)), np.ones((1, D)), wq, wk, 0.0, oracle.F64)
+    dest, sign = (j + half, 1.0) if j < half else (j - half, -1.0)
+    want_q = np.zeros(D)
+    want_q[dest] = sign * -math.sqrt(D) * wq[j]
+    want_k = np.zeros(D)
+    want_k[dest] = sign * math.sqrt(D) * wk[j]
+    np.testing.assert_allclose(q[0, 0], want_q, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(k[0, 0], want_k, rtol=0, atol=1e-14)
+
+
+def test_norm_rope_with_unit_weights_commutes_with_a_pair_rotation():
+    """With w = 1 the norm is a scalar per head and the rope (pairs sharing an
+    angle) preserves the head's norm, so normalising after the rotation gives
+    the same result; per element, the output is the rotated input over its RMS."""
+    qkv, c, s = _rope_case(6, 2, 32, 133)
+    x = oracle.widen(qkv, oracle.BF16)
+    w = np.ones(32)
+    q, k, _ = oracle.qkv_norm_rope(qkv, c, s, w, w, 0.0, oracle.BF16)
+    zq = x[:, 0, :, :16] + 1j * x[:, 0, :, 16:]
+    e = c[:, None, :16].astype(np.float64) + 1j * s[:, None, :16].astype(np.float64)
+    rms = np.sqrt(np.mean(x[:, 0] ** 2, axis=-1))[..., None]
+    zr = zq * e / rms
+    np.testing.assert_allclose(q[..., :16], zr.real, rtol=0, atol=1e-6)  # |c + i s| = 1 to float32 rounding
+    np.testing.assert_allclose(q[..., 16:], zr.imag, rtol=0, atol=1e-6)
+    assert np.all(np.isfinite(k))
+
+
+def test_norm_rope_zero_row_with_eps_is_zero():
+    qkv = np.zeros((2, 3, 1, 16))
+    q, k, _ = oracle.qkv_norm_rope(qkv, np.ones((2, 16)), np.zeros((2, 16)), np.ones(16), np.ones(16), 1e-6,
+                                   oracle.F64)
+    assert not q.any() and not k.any()
+
+
 # ---------------------------------------------------------------- grouped-query attention
 
 @pytest.mark.parametrize("H,Hkv", [(4, 2), (6, 3), (4, 1), (3, 3)])
