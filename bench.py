@@ -7,8 +7,10 @@ For a ragged multi-image workload (``--workload multi_image``) a step is one
 call of ``vitattn_forward_varlen`` over the packed batch, and the flops are
 4*H*D*sum(n_s^2) over its images.  For the prologue workload
 (``--workload rope_batched``) a step is one ``vitattn_qkv_rope`` call (packed
-QKV split + 2-D rope) and the metric is its algorithmic bytes per second
-against the measured HBM copy bandwidth.
+QKV split + 2-D rope), and for ``rope_norm_batched`` one
+``vitattn_qkv_norm_rope`` call (the same with a per-head q/k RMS norm first);
+the metric is the algorithmic bytes per second against the measured HBM copy
+bandwidth.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
@@ -53,9 +55,13 @@ METRIC = "attention fwd TFLOP/s (4·B·H·N²·D) and % of B200 dense BF16 tenso
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAK_TFLOPS = 1590.0  # the pool's earlier measurement, used only without MEASURED_PEAKS.json
 DATASHEET_PEAK_TFLOPS = 2250.0
-KERNEL_SOURCES = ["vit_bidirectional_attention_b200/csrc/fwd_kernel.cuh",
-                  "vit_bidirectional_attention_b200/csrc/ptx.cuh",
-                  "vit_bidirectional_attention_b200/csrc/rope_kernel.cuh"]
+# the device sources each kernel is compiled from (its own file and what it includes)
+_CSRC = "vit_bidirectional_attention_b200/csrc/"
+KERNEL_SOURCES = {
+    "fwd_kernel": [_CSRC + "fwd_kernel.cuh", _CSRC + "ptx.cuh"],
+    "qkv_rope_kernel": [_CSRC + "rope_kernel.cuh"],
+    "qkv_norm_rope_kernel": [_CSRC + "rope_kernel.cuh", _CSRC + "norm_rope_kernel.cuh"],
+}
 
 
 def parse():
@@ -74,9 +80,16 @@ def parse():
     return ap.parse_args()
 
 
-def kernel_hash() -> str:
+def kernel_of(workload: str) -> str:
+    """The kernel a workload's step launches."""
+    if workload in synth.PROLOGUE:
+        return "qkv_norm_rope_kernel" if synth.PROLOGUE[workload].qk_norm else "qkv_rope_kernel"
+    return "fwd_kernel"
+
+
+def kernel_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -99,7 +112,7 @@ def committed_traffic(workload: str):
     with open(path) as f:
         data = json.load(f)
     entry = data.get(workload)
-    if not entry or entry.get("kernel_hash") != kernel_hash():
+    if not entry or entry.get("kernel_hash") != kernel_hash(kernel_of(workload)):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -311,14 +324,20 @@ def run_reference(args):
 
 
 PROLOGUE_METRIC = "qkv split + 2-D rope prologue GB/s (algorithmic bytes / device time) and % of measured HBM copy bandwidth"
+PROLOGUE_NORM_METRIC = ("qkv split + q/k RMS norm + 2-D rope prologue GB/s (algorithmic bytes / device time) and % of "
+                        "measured HBM copy bandwidth")
 
 
 def run_prologue(args):
-    """The prologue workload: one vitattn_qkv_rope call per step."""
+    """The prologue workload: one vitattn_qkv_rope (or, with the q/k norm,
+    vitattn_qkv_norm_rope) call per step."""
     w = synth.PROLOGUE[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     qkv, cs, sn = synth.make_prologue(w)
+    qw, kw = synth.make_norm_weights(w.D, w.seed + 1000) if w.qk_norm else (None, None)
+    metric = PROLOGUE_NORM_METRIC if w.qk_norm else PROLOGUE_METRIC
+    entry = "vitattn_qkv_norm_rope" if w.qk_norm else "vitattn_qkv_rope"
 
     def cpu_leg(seconds, steps=1):
         # the oracle on a bounded, seeded sample of tokens; bytes scaled per token
@@ -330,7 +349,10 @@ def run_prologue(args):
             idx = np.random.Generator(np.random.PCG64(w.seed + attempt)).choice(w.T, min(n, w.T), replace=False)
             t0 = time.perf_counter()
             for _ in range(steps):
-                oracle.qkv_rope(qkv[idx], cs[idx], sn[idx], w.dtype)
+                if w.qk_norm:
+                    oracle.qkv_norm_rope(qkv[idx], cs[idx], sn[idx], qw, kw, w.eps, w.dtype)
+                else:
+                    oracle.qkv_rope(qkv[idx], cs[idx], sn[idx], w.dtype)
             dt = (time.perf_counter() - t0) / steps
             if dt >= 0.5 * seconds or n >= w.T:
                 break
@@ -345,7 +367,7 @@ def run_prologue(args):
         import oracle
 
         value, n, dt = cpu_leg(2.0, steps=max(1, args.steps or 1))
-        line = {"impl": "reference", "metric": PROLOGUE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        line = {"impl": "reference", "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world,
                 "steps": args.steps or 1, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": w.name, "tokens": w.T, "H": w.H, "D": w.D, "sample_tokens": n},
@@ -365,16 +387,23 @@ def run_prologue(args):
     hqkv = torch.from_numpy(qkv.view(np.int16).copy()).view(tdt)
     hcs, hsn = torch.from_numpy(cs), torch.from_numpy(sn)
     dqkv, dcs, dsn = (x.to(dev) for x in (hqkv, hcs, hsn))
+    hqw, hkw = (torch.from_numpy(x) for x in (qw, kw)) if w.qk_norm else (None, None)
+    dqw, dkw = (hqw.to(dev), hkw.to(dev)) if w.qk_norm else (None, None)
     q, k, v = (torch.empty((w.T, w.H, w.D), dtype=tdt, device=dev) for _ in range(3))
     stream = torch.cuda.Stream(dev)
     sh = stream.cuda_stream
     L = vitattn.lib()
 
     def step():
-        rc = L.vitattn_qkv_rope(dqkv.data_ptr(), dcs.data_ptr(), dsn.data_ptr(), q.data_ptr(), k.data_ptr(),
-                                v.data_ptr(), w.T, w.H, w.D, w.dtype, sh)
+        if w.qk_norm:
+            rc = L.vitattn_qkv_norm_rope(dqkv.data_ptr(), dcs.data_ptr(), dsn.data_ptr(), dqw.data_ptr(),
+                                         dkw.data_ptr(), w.eps, q.data_ptr(), k.data_ptr(), v.data_ptr(), w.T, w.H,
+                                         w.D, w.dtype, sh)
+        else:
+            rc = L.vitattn_qkv_rope(dqkv.data_ptr(), dcs.data_ptr(), dsn.data_ptr(), q.data_ptr(), k.data_ptr(),
+                                    v.data_ptr(), w.T, w.H, w.D, w.dtype, sh)
         if rc:
-            raise vitattn.VitAttnError(rc, "vitattn_qkv_rope")
+            raise vitattn.VitAttnError(rc, entry)
 
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     sampler.start()
@@ -416,13 +445,19 @@ def run_prologue(args):
 
     # end to end through the Python entry, host copies on the same stream
     hqkv_p, hcs_p, hsn_p = (x.pin_memory() for x in (hqkv, hcs, hsn))
+    hqw_p, hkw_p = (hqw.pin_memory(), hkw.pin_memory()) if w.qk_norm else (None, None)
     hq, hk, hv = (torch.empty((w.T, w.H, w.D), dtype=tdt).pin_memory() for _ in range(3))
 
     def e2e_step():
         dqkv.copy_(hqkv_p, non_blocking=True)
         dcs.copy_(hcs_p, non_blocking=True)
         dsn.copy_(hsn_p, non_blocking=True)
-        oq, ok, ov = vitattn.qkv_rope(dqkv, dcs, dsn, stream=stream)
+        if w.qk_norm:
+            dqw.copy_(hqw_p, non_blocking=True)
+            dkw.copy_(hkw_p, non_blocking=True)
+            oq, ok, ov = vitattn.qkv_norm_rope(dqkv, dcs, dsn, dqw, dkw, w.eps, stream=stream)
+        else:
+            oq, ok, ov = vitattn.qkv_rope(dqkv, dcs, dsn, stream=stream)
         hq.copy_(oq, non_blocking=True)
         hk.copy_(ok, non_blocking=True)
         hv.copy_(ov, non_blocking=True)
@@ -451,23 +486,23 @@ def run_prologue(args):
             value, n, dt = cpu_leg(args.cpu_seconds)
             cpu = {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
                    "sample": f"{n} of {w.T} tokens (seeded), numpy fp64, {dt:.1f} s"}
-        in_bytes = 3 * w.T * w.H * w.D * 2 + 2 * w.T * w.D * 4
+        in_bytes = 3 * w.T * w.H * w.D * 2 + 2 * w.T * w.D * 4 + (8 * w.D if w.qk_norm else 0)
         result = {
-            "metric": PROLOGUE_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "metric": metric, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
             "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": synth.DTYPE_NAMES[w.dtype],
             "data": "synthetic (seeded normals; 2-D rope tables of the patch grid)",
             "config": {"workload": w.name, "images": w.images, "grid": list(w.grid), "tokens": w.T, "H": w.H,
-                       "D": w.D, "global_batch": w.images * world,
+                       "D": w.D, "qk_norm": w.qk_norm, "global_batch": w.images * world,
                        "l2": f"{w.io_bytes / 2**20:.0f} MiB moved per step > 126 MiB L2, no flush",
                        "bytes_per_step": w.io_bytes},
             "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s", "frac": per_gpu / peak,
                          "traffic": committed_traffic(w.name),
                          "peak_source": "measured copy bandwidth, MEASURED_PEAKS.json" if peaks else "fallback",
-                         "kernel": "vitattn::qkv_rope_kernel", "algorithmic_bytes_per_launch": w.io_bytes},
+                         "kernel": "vitattn::" + kernel_of(w.name), "algorithmic_bytes_per_launch": w.io_bytes},
             "e2e": {"value": w.io_bytes * n_e2e * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": 3 * w.T * w.H * w.D * 2,
-                    "ms_per_step": e2e_ms / n_e2e, "entry": "qkv_rope + stream copies"},
+                    "ms_per_step": e2e_ms / n_e2e, "entry": entry[len("vitattn_"):] + " + stream copies"},
             "gpu_launches": steps,
             "clocks": clocks,
             "cpu_baseline": cpu,

@@ -24,6 +24,7 @@
  *   vitattn_forward_gqa      grouped-query attention (fewer key/value heads)
  *   vitattn_forward_ext      Lq != Lk, aligned causal mask, log-sum-exp output
  *   vitattn_qkv_rope         the prologue: packed QKV split + rotary embedding
+ *   vitattn_qkv_norm_rope    the same with a per-head q/k RMS norm before the rope
  *   vitattn_forward_host     vitattn_forward from host buffers (copies enqueued)
  *   ..._checked, ..._check_args*, vitattn_strerror, vitattn_last_cuda_error,
  *   vitattn_version, vitattn_launches_per_call: synchronising variants for
@@ -93,7 +94,7 @@ enum vitattn_status {
     VITATTN_ERR_ALIAS = -6,   /* out overlaps q, k or v */
     VITATTN_ERR_CUDA = -7,    /* the CUDA runtime or driver returned an error */
     VITATTN_ERR_TIMEOUT = -8, /* a bounded in-kernel wait ran out (checked entry only) */
-    VITATTN_ERR_SCALE = -9,   /* scale is NaN or infinite */
+    VITATTN_ERR_SCALE = -9,   /* scale is NaN or infinite (or eps negative / not finite) */
     VITATTN_ERR_DEVICE = -10, /* the current device is not an sm_100 GPU */
     VITATTN_ERR_RANGE = -11,  /* a bf16 V value has |v| >= 65536 (checked entry only) */
     VITATTN_ERR_SEQLENS = -12 /* cu_seqlens does not start at 0 or decreases somewhere */
@@ -256,6 +257,39 @@ VITATTN_API int vitattn_qkv_rope(const void* qkv, const float* cos_table, const 
 VITATTN_API int vitattn_check_args_qkv_rope(const void* qkv, const float* cos_table, const float* sin_table,
                                             const void* q, const void* k, const void* v, int64_t T, int64_t H,
                                             int64_t D, int dtype);
+
+/*
+ * vitattn_qkv_norm_rope -- the prologue with a per-head RMS norm of q and k
+ * ahead of the rotary embedding, in one pass.
+ * Source: inferencelayer "src/vision_gpu.rs", GLM_QKV_QKNORM_ROPE and its doc
+ * (GLM-OCR vision tower: split the packed qkv, normalise each head's q and k
+ * row over its head_dim elements with a per-element weight, BEFORE the rope;
+ * then the rope of vitattn_qkv_rope; v passes through).
+ *   qkv, cos_table, sin_table, q, k, v, T, H, D, dtype  as for
+ *             vitattn_qkv_rope.
+ *   q_norm_w, k_norm_w  device pointers, [D] float32 each, 16-byte aligned:
+ *             the weights of the q norm and of the k norm (one vector for
+ *             all heads).  They must not overlap an output.
+ *   eps       finite, >= 0 (else VITATTN_ERR_SCALE).  With eps = 0 a head
+ *             row of zeros has no defined norm and its output is NaN.
+ * Per token t, head h, x = q or k and its weight w:
+ *     y[d]  = x[d] / sqrt(mean_e x[e]^2 + eps) * w[d],
+ *     x'[d] = y[d] * cos[t,d] + r[d] * sin[t,d],
+ *     r[d]  = -y[d + D/2] (d < D/2),  y[d - D/2] (d >= D/2),
+ * computed in f32 (IEEE square root and divide) and rounded once to `dtype`;
+ * v is copied bit for bit.  Enqueues one kernel on `stream`; errors as for
+ * vitattn_forward.
+ */
+VITATTN_API int vitattn_qkv_norm_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                                      const float* q_norm_w, const float* k_norm_w, float eps, void* q, void* k,
+                                      void* v, int64_t T, int64_t H, int64_t D, int dtype,
+                                      vitattn_stream_t stream);
+
+/* The argument checks of vitattn_qkv_norm_rope alone (no CUDA call). */
+VITATTN_API int vitattn_check_args_qkv_norm_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                                                 const float* q_norm_w, const float* k_norm_w, float eps,
+                                                 const void* q, const void* k, const void* v, int64_t T,
+                                                 int64_t H, int64_t D, int dtype);
 
 /*
  * vitattn_forward_host -- the same operation from HOST buffers: enqueues the

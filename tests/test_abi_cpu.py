@@ -167,6 +167,43 @@ def test_rope_argument_errors(kw, code):
     assert check_rope(**kw) == code
 
 
+def check_norm_rope(**kw):
+    T, H, D = kw.get("T", 64), kw.get("H", 2), kw.get("D", 64)
+    row = H * D * 2
+    # disjoint fake regions: qkv | cos | sin | q | k | v | q_norm_w | k_norm_w
+    a = dict(qkv=A, cos=A + 3 * row * T, sin=A + 3 * row * T + T * D * 4, q=A + 3 * row * T + 2 * T * D * 4,
+             eps=1e-6, T=T, H=H, D=D, dtype=vitattn.BF16)
+    a["k"] = a["q"] + row * T
+    a["v"] = a["k"] + row * T
+    a["qw"] = a["v"] + row * T
+    a["kw"] = a["qw"] + D * 4
+    a.update(kw)
+    return vitattn.check_args_qkv_norm_rope(a["qkv"], a["cos"], a["sin"], a["qw"], a["kw"], a["eps"], a["q"], a["k"],
+                                            a["v"], a["T"], a["H"], a["D"], a["dtype"])
+
+
+def test_norm_rope_valid_arguments_pass():
+    assert check_norm_rope() == 0
+    assert check_norm_rope(D=128, dtype=vitattn.F16, eps=0.0) == 0
+    assert check_norm_rope(kw=A) == 0                  # weights are read-only inputs: sharing qkv's memory is fine
+
+
+V_END = A + 3 * 256 * 64 + 2 * 64 * 64 * 4 + 3 * 256 * 64   # one past v in the default layout
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(qw=0), -1), (dict(kw=0), -1), (dict(qkv=0), -1),
+    (dict(T=0), -2), (dict(D=60), -3), (dict(dtype=3), -4),
+    (dict(qw=V_END + 4), -5), (dict(kw=V_END + 8), -5),
+    (dict(eps=-1e-6), -9), (dict(eps=float("nan")), -9), (dict(eps=float("inf")), -9),
+    (dict(qw=V_END - 64), -6),                         # overlaps the tail of v
+    (dict(kw=A + 3 * 256 * 64 + 2 * 64 * 64 * 4 + 32), -6),   # inside q
+    (dict(q=A + 16), -6),                              # the rope checks still apply
+])
+def test_norm_rope_argument_errors(kw, code):
+    assert check_norm_rope(**kw) == code
+
+
 # ---------------------------------------------------------------- grouped-query attention
 
 def check_gqa(**kw):

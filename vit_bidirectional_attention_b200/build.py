@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libvitattn.so")
 SOURCES = [os.path.join(CSRC, "vitattn.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fwd_kernel.cuh", "ptx.cuh")] + [
+DEPS = SOURCES + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(INCLUDE, "vitattn.h")]
 
 NVCC_FLAGS = [

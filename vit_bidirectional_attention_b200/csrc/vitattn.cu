@@ -14,6 +14,7 @@
 #include "vitattn.h"
 
 #include "fwd_kernel.cuh"
+#include "norm_rope_kernel.cuh"
 #include "rope_kernel.cuh"
 
 namespace {
@@ -164,6 +165,24 @@ int check_args_rope(const void* qkv, const float* cs, const float* sn, const voi
         for (int j = 0; j < i; ++j)
             if (overlaps(outs[i], outs[j], out_bytes)) return VITATTN_ERR_ALIAS;
     }
+    return VITATTN_OK;
+}
+
+// The prologue with q/k RMS norm: the rope checks, plus two [D] f32 weight
+// vectors (16-byte aligned, not overlapping an output) and a finite eps >= 0.
+int check_args_norm_rope(const void* qkv, const float* cs, const float* sn, const float* qw, const float* kw,
+                         float eps, const void* q, const void* k, const void* v, int64_t T, int64_t H,
+                         int64_t D, int dtype) {
+    int rc = check_args_rope(qkv, cs, sn, q, k, v, T, H, D, dtype);
+    if (rc) return rc;
+    if (!qw || !kw) return VITATTN_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(qw) | reinterpret_cast<uintptr_t>(kw)) & 15u) return VITATTN_ERR_ALIGN;
+    if (!std::isfinite(eps) || eps < 0.f) return VITATTN_ERR_SCALE;
+    const uint64_t out_bytes = (uint64_t)H * (uint64_t)D * 2u * (uint64_t)T, w_bytes = (uint64_t)D * 4u;
+    const void* outs[3] = {q, k, v};
+    for (int i = 0; i < 3; ++i)
+        if (overlaps2(outs[i], out_bytes, qw, w_bytes) || overlaps2(outs[i], out_bytes, kw, w_bytes))
+            return VITATTN_ERR_ALIAS;
     return VITATTN_OK;
 }
 
@@ -453,6 +472,33 @@ int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void
     return VITATTN_OK;
 }
 
+// The prologue with q/k RMS norm: as launch_rope, with a grid of the blocks
+// that are resident at once (kNormRopeBlocksPerSm per SM).
+int launch_norm_rope(const void* qkv, const float* cs, const float* sn, const float* qw, const float* kw,
+                     float eps, void* q, void* k, void* v, int64_t T, int64_t H, int64_t D, int dtype,
+                     cudaStream_t stream) {
+    int rc = check_args_norm_rope(qkv, cs, sn, qw, kw, eps, q, k, v, T, H, D, dtype);
+    if (rc) return rc;
+    int num_sms = 0;
+    rc = device_info(&num_sms);
+    if (rc) return rc;
+    const uint64_t items = (uint64_t)T * (uint64_t)((H + vitattn::kRopeHeadsPerWarp - 1) / vitattn::kRopeHeadsPerWarp);
+    const uint64_t per_block = (uint64_t)(vitattn::kRopeThreads / 32);
+    const uint64_t want = (items + per_block - 1) / per_block;
+    const unsigned grid =
+        (unsigned)std::min<uint64_t>(want, (uint64_t)num_sms * (uint64_t)vitattn::kNormRopeBlocksPerSm);
+    auto qkv8 = static_cast<const uint8_t*>(qkv);
+    auto q8 = static_cast<uint8_t*>(q), k8 = static_cast<uint8_t*>(k), v8 = static_cast<uint8_t*>(v);
+    long long TT = (long long)T;
+    int HH = (int)H, DD = (int)D;
+    void* args[12] = {&qkv8, &cs, &sn, &qw, &kw, &eps, &q8, &k8, &v8, &TT, &HH, &DD};
+    const void* fn = dtype == VITATTN_BF16 ? reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true>)
+                                           : reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false>);
+    cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(vitattn::kRopeThreads), args, 0, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return VITATTN_OK;
+}
+
 // Launch (through `go`), synchronise, and read the kernel's status words.
 template <class Go>
 int checked_run(cudaStream_t stream, Go go) {
@@ -634,6 +680,19 @@ int vitattn_check_args_qkv_rope(const void* qkv, const float* cos_table, const f
     return check_args_rope(qkv, cos_table, sin_table, q, k, v, T, H, D, dtype);
 }
 
+int vitattn_qkv_norm_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                          const float* q_norm_w, const float* k_norm_w, float eps, void* q, void* k, void* v,
+                          int64_t T, int64_t H, int64_t D, int dtype, vitattn_stream_t stream) {
+    return launch_norm_rope(qkv, cos_table, sin_table, q_norm_w, k_norm_w, eps, q, k, v, T, H, D, dtype,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int vitattn_check_args_qkv_norm_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                                     const float* q_norm_w, const float* k_norm_w, float eps, const void* q,
+                                     const void* k, const void* v, int64_t T, int64_t H, int64_t D, int dtype) {
+    return check_args_norm_rope(qkv, cos_table, sin_table, q_norm_w, k_norm_w, eps, q, k, v, T, H, D, dtype);
+}
+
 int vitattn_forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq,
                          void* dk, void* dv, void* dout, int64_t B, int64_t N, int64_t H,
                          int64_t D, float scale, int dtype, vitattn_stream_t stream) {
@@ -671,7 +730,7 @@ const char* vitattn_strerror(int status) {
         case VITATTN_ERR_ALIAS: return "out overlaps q, k or v";
         case VITATTN_ERR_CUDA: return "CUDA error (see vitattn_last_cuda_error)";
         case VITATTN_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
-        case VITATTN_ERR_SCALE: return "scale must be finite";
+        case VITATTN_ERR_SCALE: return "scale must be finite (eps: finite and >= 0)";
         case VITATTN_ERR_DEVICE: return "the current device is not an sm_100 GPU";
         case VITATTN_ERR_SEQLENS: return "cu_seqlens must start at 0 and never decrease";
         case VITATTN_ERR_RANGE: return "a bf16 V value has magnitude >= 65536, outside the f16 P.V product's range";

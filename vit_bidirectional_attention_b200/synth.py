@@ -219,6 +219,8 @@ class PrologueWorkload:
     D: int
     dtype: int
     index: int = 0
+    qk_norm: bool = False   # per-head RMS norm of q and k before the rope
+    eps: float = 1e-6
 
     @property
     def seed(self) -> int:
@@ -230,8 +232,9 @@ class PrologueWorkload:
 
     @property
     def io_bytes(self) -> int:
-        """qkv read, cos/sin read, q/k/v written: each once."""
-        return 2 * (3 * self.T * self.H * self.D * 2) + 2 * self.T * self.D * 4
+        """qkv read, cos/sin read, q/k/v written: each once (plus the two
+        [D] f32 norm weights when ``qk_norm``)."""
+        return 2 * (3 * self.T * self.H * self.D * 2) + 2 * self.T * self.D * 4 + (8 * self.D if self.qk_norm else 0)
 
 
 PROLOGUE = {
@@ -239,6 +242,8 @@ PROLOGUE = {
     for w in (
         # the QKV of the batched workload: 32 images of 32 x 32 patches, 16 heads, D = 64
         PrologueWorkload("rope_batched", 32, (32, 32), 16, 64, BF16, index=6),
+        # the same, with the q/k RMS norm ahead of the rope (the GLM-OCR tower's prologue)
+        PrologueWorkload("rope_norm_batched", 32, (32, 32), 16, 64, BF16, index=9, qk_norm=True),
     )
 }
 
@@ -248,6 +253,14 @@ def make_prologue(w: PrologueWorkload):
     qkv = make_qkv_packed(w.T, w.H, w.D, w.dtype, seed=w.seed)
     cs, sn = rope_tables_2d(w.grid[0], w.grid[1], w.D)
     return qkv, np.tile(cs, (w.images, 1)), np.tile(sn, (w.images, 1))
+
+
+def make_norm_weights(D: int, seed: int):
+    """(q_norm_w, k_norm_w) float32 ``[D]`` each: 1 + 0.25 * N(0, 1), the
+    spread of a trained RMS-norm weight around its initial value of one."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    w = 1.0 + 0.25 * rng.standard_normal(size=(2, D))
+    return w[0].astype(np.float32), w[1].astype(np.float32)
 
 
 def make_qkv_packed(T: int, H: int, D: int, dtype: int, seed: int, std: float = 1.0):

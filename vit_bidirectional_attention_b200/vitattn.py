@@ -75,6 +75,9 @@ def lib() -> ctypes.CDLL:
         rope = [p, p, p, p, p, p, i64, i64, i64, i32]
         L.vitattn_qkv_rope.argtypes = rope + [p]
         L.vitattn_check_args_qkv_rope.argtypes = rope
+        norm_rope = [p, p, p, p, p, f32, p, p, p, i64, i64, i64, i32]
+        L.vitattn_qkv_norm_rope.argtypes = norm_rope + [p]
+        L.vitattn_check_args_qkv_norm_rope.argtypes = norm_rope
         L.vitattn_strerror.argtypes = [i32]
         L.vitattn_strerror.restype = ctypes.c_char_p
         for f in (L.vitattn_forward, L.vitattn_forward_checked, L.vitattn_test_forward_flags,
@@ -84,7 +87,8 @@ def lib() -> ctypes.CDLL:
                   L.vitattn_check_args_varlen, L.vitattn_qkv_rope, L.vitattn_check_args_qkv_rope,
                   L.vitattn_forward_gqa, L.vitattn_forward_gqa_checked, L.vitattn_test_forward_gqa_flags,
                   L.vitattn_check_args_gqa, L.vitattn_forward_ext, L.vitattn_forward_ext_checked,
-                  L.vitattn_test_forward_ext_flags, L.vitattn_check_args_ext):
+                  L.vitattn_test_forward_ext_flags, L.vitattn_check_args_ext, L.vitattn_qkv_norm_rope,
+                  L.vitattn_check_args_qkv_norm_rope):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -289,6 +293,57 @@ def qkv_rope(qkv, cos, sin, stream=None):
                           v.data_ptr(), T, H, D, dtype, handle)
     if rc != 0:
         raise VitAttnError(rc, "vitattn_qkv_rope")
+    return q, k, v
+
+
+def check_args_qkv_norm_rope(qkv, cos, sin, q_norm_w, k_norm_w, eps, q, k, v, T, H, D, dtype) -> int:
+    """Status the normed prologue's argument checks give (pointers as ints); no CUDA call."""
+    return int(lib().vitattn_check_args_qkv_norm_rope(qkv, cos, sin, q_norm_w, k_norm_w, float(eps), q, k, v,
+                                                       T, H, D, dtype))
+
+
+def qkv_norm_rope_ptr(qkv, cos, sin, q_norm_w, k_norm_w, eps, q, k, v, T, H, D, dtype, stream=0) -> int:
+    """Raw normed prologue call on device pointers (ints); returns the status."""
+    return int(lib().vitattn_qkv_norm_rope(qkv, cos, sin, q_norm_w, k_norm_w, float(eps), q, k, v, T, H, D,
+                                           dtype, stream))
+
+
+def qkv_norm_rope(qkv, cos, sin, q_norm_w, k_norm_w, eps, stream=None):
+    """Split a packed QKV projection, RMS-normalise each head's q and k row
+    (weights ``q_norm_w``, ``k_norm_w``: contiguous float32 ``[D]`` CUDA
+    tensors; ``eps`` >= 0), then rotate q and k.  Other arguments and the
+    result as for :func:`qkv_rope`."""
+    import torch
+
+    if qkv.dim() < 4 or qkv.shape[-3] != 3:
+        raise ValueError("qkv must be [..., 3, H, D]")
+    ts = (qkv, cos, sin, q_norm_w, k_norm_w)
+    if not all(t.is_cuda for t in ts):
+        raise ValueError("qkv, cos, sin and the norm weights must be CUDA tensors")
+    if not all(t.is_contiguous() for t in ts):
+        raise ValueError("qkv, cos, sin and the norm weights must be contiguous")
+    if any(t.dtype != torch.float32 for t in ts[1:]):
+        raise TypeError("cos, sin and the norm weights must be float32")
+    dtype = _dtype_code(qkv)
+    lead = tuple(qkv.shape[:-3])
+    H, D = qkv.shape[-2], qkv.shape[-1]
+    T = 1
+    for n in lead:
+        T *= n
+    if tuple(cos.shape) != (T, D) or tuple(sin.shape) != (T, D):
+        raise ValueError("cos and sin must be [T, D] with T the token count of qkv")
+    if tuple(q_norm_w.shape) != (D,) or tuple(k_norm_w.shape) != (D,):
+        raise ValueError("the norm weights must be [D]")
+    q, k, v = (torch.empty(lead + (H, D), dtype=qkv.dtype, device=qkv.device) for _ in range(3))
+    if stream is None:
+        stream = torch.cuda.current_stream(qkv.device)
+    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    with torch.cuda.device(qkv.device):
+        rc = qkv_norm_rope_ptr(qkv.data_ptr(), cos.data_ptr(), sin.data_ptr(), q_norm_w.data_ptr(),
+                               k_norm_w.data_ptr(), eps, q.data_ptr(), k.data_ptr(), v.data_ptr(), T, H, D,
+                               dtype, handle)
+    if rc != 0:
+        raise VitAttnError(rc, "vitattn_qkv_norm_rope")
     return q, k, v
 
 
