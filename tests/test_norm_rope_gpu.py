@@ -4,19 +4,20 @@
 row with a per-element weight, then rotate), against the fp64 oracle
 ``qkv_norm_rope``.
 
-Error bound.  The kernel works in f32:
-- the head's sum of squares, with at most 8 roundings along any path (4 per
-  lane, then a 5-level butterfly), all terms positive: relative error <= 8u,
-  with u = 2^-24;
-- the division by D, the addition of eps, the square root and the reciprocal:
-  about 3.5u more on the inverse root, which totals <= 8u;
-- y = x*inv*w and its rotation partner: two more roundings each;
-- one product with sin, then one fma with cos.
+Error bound.  The kernel computes x' = inv * (x*A + p*B) in f32, with
+A = w*cos, B = sign*w_p*sin formed once per token and inv the inverse root:
+- the head's sum of squares takes at most 9 roundings along any path (4 per
+  lane, then a butterfly of up to 5 levels), and all its terms are positive:
+  relative error <= 9u, with u = 2^-24;
+- the mean plus eps is one fma with 1/D (2u), and rsqrtf adds at most 2 ulp
+  (4u), so inv is within about 10u;
+- A, B and p*B take one rounding each, then the fma and the product with inv
+  take one more each.
 Every q/k element must therefore lie within one unit in the last place (of
-the storage dtype) of the exact value, plus 2^-19 * (|y*c| + |y_p*s|).  The
-2^-19 allows 32u, about three times the 11u the steps above add up to.  At
-least 99% of the elements must be the exact round-to-nearest result, and v
-must be a bit-exact copy.
+the storage dtype) of the exact value, plus 2^-19 * (|y*c| + |y_p*s|), where
+y is the normed row.  The 2^-19 allows 32u, about twice the ~15u the steps
+above add up to.  At least 99% of the elements must be the exact
+round-to-nearest result, and v must be a bit-exact copy.
 """
 import numpy as np
 import pytest
