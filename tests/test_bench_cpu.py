@@ -98,3 +98,70 @@ def test_library_rebuild_tracks_every_kernel_header():
     headers = {os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith(".cuh")}
     assert headers <= set(build.DEPS)
     assert os.path.join(ROOT, "include", "vitattn.h") in build.DEPS
+
+
+class FakeClock:
+    """A device timeline: launches advance it; events read it when recorded."""
+
+    def __init__(self):
+        self.now = 0.0
+        self.log = []
+
+
+def fake_event_cls(clock):
+    class Event:
+        def __init__(self, enable_timing=False):
+            assert enable_timing
+            self.t = None
+
+        def record(self, stream):
+            assert stream == "s"
+            self.t = clock.now
+            clock.log.append("event")
+
+        def synchronize(self):
+            assert self.t is not None
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    return Event
+
+
+@pytest.mark.parametrize("steps", [1, 7])
+def test_timed_launches_without_flush_times_the_whole_region(steps):
+    clock = FakeClock()
+
+    def step():
+        clock.now += 2.0
+        clock.log.append("kernel")
+
+    ms = bench.timed_launches(step, steps, "s", fake_event_cls(clock))
+    assert ms == 2.0 * steps
+    assert clock.log == ["event"] + ["kernel"] * steps + ["event"]
+
+
+@pytest.mark.parametrize("steps", [1, 7])
+def test_timed_launches_with_flush_times_only_the_launches(steps):
+    """The flush runs before every launch and its time is left out: only the
+    kernels' own intervals are summed."""
+    clock = FakeClock()
+
+    def step():
+        clock.now += 2.0
+        clock.log.append("kernel")
+
+    def flush():
+        clock.now += 40.0
+        clock.log.append("flush")
+
+    ms = bench.timed_launches(step, steps, "s", fake_event_cls(clock), flush=flush)
+    assert ms == 2.0 * steps
+    assert clock.log == ["flush", "event", "kernel", "event"] * steps
+
+
+def test_flush_buffer_exceeds_l2():
+    assert bench.L2_FLUSH_BYTES > bench.L2_BYTES
+    small = [n for n, w in synth.WORKLOADS.items() if w.io_bytes <= bench.L2_BYTES]
+    assert set(small) >= {"tiny", "small_vit", "doc_page"}
+    assert "batched" not in small and "high_res" not in small
