@@ -14,7 +14,7 @@
 //     A[d] = w[d] * cos[d],  B[d] = sign(d) * w[p(d)] * sin[d],
 // with p the rotation partner d +- D/2 and inv = 1/sqrt(mean x^2 + eps): A
 // and B are formed once per token (from the weights, re-read from L1, and
-// the token's table row) and serve all its heads, leaving three multiplies
+// the token's table row) and serve all its heads, leaving two multiplies
 // and an fma per element.  The head's sum of squares is an xor butterfly
 // over the lanes the head occupies (lanes past D/4 inside that power of two
 // hold zeros; a + b == b + a, so every lane ends with the same sum); the
