@@ -711,7 +711,7 @@ def main():
         peak_note = "measured burst dense bf16 (cuBLAS 8192^3), MEASURED_PEAKS.json"
     else:
         peak = FALLBACK_PEAK_TFLOPS
-        peak_note = "fallback 1.59 PFLOP/s (pool's earlier measurement)"
+        peak_note = "fallback 1.59 PFLOP/s (an earlier B200 measurement)"
     if w.dtype == synth.F16:
         peak_note += "; f16 runs at the bf16 rate (same nominal dense figure)"
 
