@@ -294,7 +294,11 @@ VITATTN_API int vitattn_check_args_qkv_norm_rope(const void* qkv, const float* c
 /*
  * vitattn_forward_host -- the same operation from HOST buffers: enqueues the
  * copies hq->dq, hk->dk, hv->dv, the kernel, and dout->hout, in that order,
- * on `stream`, and returns without synchronising.  The caller synchronises
+ * on `stream`, and returns without synchronising.  Source: hanzo-ml
+ * "src/vulkan_backend.rs", `flash_attn` (the host-data convenience form of
+ * `flash_attn_gpu`: upload the inputs, run the device entry, read the
+ * output back).  Here the caller supplies the device staging buffers, so
+ * the library still allocates nothing.  The caller synchronises
  * the stream before reading hout.  Host buffers should be pinned
  * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous; the
  * device buffers dq, dk, dv, dout are caller-owned staging with the same

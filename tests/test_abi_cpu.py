@@ -251,3 +251,18 @@ def test_ext_valid_arguments_pass():
 ])
 def test_ext_argument_errors(kw, code):
     assert check_ext(**kw) == code
+
+
+def test_every_compute_entry_cites_the_passage_that_defines_it():
+    """Each entry that launches work documents its operation with a reference
+    to the page (by source path) that defines it."""
+    text = open(HEADER).read()
+    compute = {"vitattn_forward", "vitattn_forward_ext", "vitattn_forward_gqa", "vitattn_forward_varlen",
+               "vitattn_qkv_rope", "vitattn_qkv_norm_rope", "vitattn_forward_host"}
+    seen = set()
+    for m in re.finditer(r"/\*(.*?)\*/\s*VITATTN_API[^;(]*?\b(vitattn_\w+)\s*\(", text, re.S):
+        comment, name = m.group(1), m.group(2)
+        if name in compute:
+            assert re.search(r"src/[\w/]+\.rs", comment), f"{name}: no source citation"
+            seen.add(name)
+    assert seen == compute
