@@ -81,6 +81,20 @@ def parse():
     return ap.parse_args()
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first entry of /proc/cpuinfo), for the CPU baseline."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
 def timed_launches(step, steps: int, stream, event_cls, flush=None) -> float:
     """Device milliseconds of ``steps`` launches of ``step`` on ``stream``.
 
@@ -259,7 +273,7 @@ def cpu_baseline(w, q, k, v, seconds: float):
             break
         n = int(min(total_rows, max(2 * n, len(rows) * seconds / max(dt, 1e-6))))
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s",
-            "cores": oracle.num_threads(), "kind": "oracle",
+            "cores": oracle.num_threads(), "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"{len(rows)} of {total_rows} output rows (seeded), fp64, "
                       f"{dt:.1f} s on {oracle.num_threads()} threads"}
 
@@ -340,7 +354,7 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(shape_config(w), workload=args.workload, input_dtype=synth.DTYPE_NAMES[w.dtype],
                        scale=w.scale, sample_rows_per_step=n_rows),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "cpu_model": cpu_model(),
                          "kind": "oracle",
                          "sample": f"{n_rows} of {total_rows} output rows per step (seeded)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -397,7 +411,7 @@ def run_prologue(args):
                 "steps": args.steps or 1, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": w.name, "tokens": w.T, "H": w.H, "D": w.D, "sample_tokens": n},
-                "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "cpu_model": cpu_model(), "kind": "oracle",
                                  "sample": f"{n} of {w.T} tokens (seeded), numpy fp64"},
                 "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -510,7 +524,7 @@ def run_prologue(args):
             import oracle
 
             value, n, dt = cpu_leg(args.cpu_seconds)
-            cpu = {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            cpu = {"value": value, "unit": "GB/s", "cores": oracle.num_threads(), "cpu_model": cpu_model(), "kind": "oracle",
                    "sample": f"{n} of {w.T} tokens (seeded), numpy fp64, {dt:.1f} s"}
         in_bytes = 3 * w.T * w.H * w.D * 2 + 2 * w.T * w.D * 4 + (8 * w.D if w.qk_norm else 0)
         result = {

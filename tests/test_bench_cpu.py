@@ -41,6 +41,7 @@ def test_reference_arm_prints_one_contract_line(workload, unit):
     assert d["config"]["workload"] == workload and d["dtype"] == "f64"
     cpu = d["cpu_baseline"]
     assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] == d["value"] and cpu["sample"]
+    assert cpu["cpu_model"] and cpu["cpu_model"] != "unknown"
     assert d["e2e"] == {"value": d["value"], "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
