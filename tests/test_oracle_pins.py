@@ -503,6 +503,24 @@ def test_norm_rope_with_unit_weights_commutes_with_a_pair_rotation():
     assert np.all(np.isfinite(k))
 
 
+def test_norm_rope_hand_fixture():
+    """D = 4 by hand.  q = (1, 2, 3, 4): mean square 30/4 = 7.5, so with
+    weights (2, 1, 1, 3) the normed row is (2, 2, 3, 12)/sqrt(7.5); the quarter
+    turn on pair 0 (angle pi/2) and none on pair 1 then give
+    (-3, 2, 2, 12)/sqrt(7.5).  k = (5, 6, 7, 8) with unit weights and eps = 0:
+    mean square 174/4 = 43.5, output (-7, 6, 5, 8)/sqrt(43.5)."""
+    qkv = np.zeros((1, 3, 1, 4))
+    qkv[0, 0, 0] = [1, 2, 3, 4]
+    qkv[0, 1, 0] = [5, 6, 7, 8]
+    qkv[0, 2, 0] = [9, 10, 11, 12]
+    c = np.array([[0.0, 1.0, 0.0, 1.0]])
+    s = np.array([[1.0, 0.0, 1.0, 0.0]])
+    q, k, v = oracle.qkv_norm_rope(qkv, c, s, np.array([2.0, 1.0, 1.0, 3.0]), np.ones(4), 0.0, oracle.F64)
+    np.testing.assert_allclose(q[0, 0], np.array([-3.0, 2.0, 2.0, 12.0]) / math.sqrt(7.5), rtol=1e-15, atol=0)
+    np.testing.assert_allclose(k[0, 0], np.array([-7.0, 6.0, 5.0, 8.0]) / math.sqrt(43.5), rtol=1e-15, atol=0)
+    assert v[0, 0].tolist() == [9.0, 10.0, 11.0, 12.0]
+
+
 def test_norm_rope_zero_row_with_eps_is_zero():
     qkv = np.zeros((2, 3, 1, 16))
     q, k, _ = oracle.qkv_norm_rope(qkv, np.ones((2, 16)), np.zeros((2, 16)), np.ones(16), np.ones(16), 1e-6,
