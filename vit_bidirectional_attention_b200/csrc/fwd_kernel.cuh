@@ -640,7 +640,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 for (int m = 0; m < 3; ++m)
                     ptx::prefetch_tensormap(&p.maps[m][width_class(chunk_width(DP, c))]);
             int r = 0;         // K/V ring entries issued so far (K_j, V_j of each item in turn)
-            int q_last[2] = {-1, -1};  // last item whose Q tile t was issued
+            // last item whose Q tile 0 / tile 1 was issued (two scalars rather than an
+            // array indexed by the tile, which would live in local memory)
+            int q_last0 = -1, q_last1 = -1;
             bool ok = true;
             for (int k = 0; k < n_my && ok; ++k) {
                 const Item it = item_of((int)blockIdx.x + k * (int)gridDim.x);
@@ -660,7 +662,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                                          &p.maps[0][width_class(chunk_width(DP, c))], chunk_col(DP, c),
                                          it.h, it.tok0 + it.q0 + t * kTileRows, it.b,
                                          bar(kBarQFull + 2 * qb + t));
-                    q_last[t] = k;
+                    if (t == 0) q_last0 = k;
+                    else q_last1 = k;
                 }
 
                 for (int j = 0; j < nkb && ok; ++j) {
@@ -688,9 +691,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 // waited for).  The last fill of each buffer or slot is its latest
                 // phase, so its parity is unambiguous whether or not it was consumed.
                 const uint64_t drain_ns = 200000000ull;
-                for (int t = 0; t < T; ++t)
-                    for (int k = q_last[t]; k >= 0 && k > q_last[t] - NQ; --k)
+                for (int t = 0; t < T; ++t) {
+                    const int q_last = t == 0 ? q_last0 : q_last1;
+                    for (int k = q_last; k >= 0 && k > q_last - NQ; --k)
                         wait_drain(bar(kBarQFull + 2 * (k % NQ) + t), (uint32_t)(k / NQ) & 1u, drain_ns);
+                }
                 for (int idx = r - 1; idx >= 0 && idx >= r - kStages; --idx) {
                     if ((p.flags & kFlagSkipFirstVLoad) && idx == 1) continue;
                     wait_drain(bar(kBarKvFull + idx % kStages), (uint32_t)(idx / kStages) & 1u,
