@@ -50,7 +50,7 @@ import numpy as np  # noqa: E402
 
 from vit_bidirectional_attention_b200 import ranks, synth  # noqa: E402
 
-DEFAULT_WORKLOAD = "batched"
+DEFAULT_WORKLOAD = "high_res"
 METRIC = "attention fwd TFLOP/s (4·B·H·N²·D) and % of B200 dense BF16 tensor peak"
 L2_BYTES = 126 * 1024 * 1024
 L2_FLUSH_BYTES = 256 * 1024 * 1024  # written before each timed launch when the inputs fit in L2
@@ -447,12 +447,20 @@ def run_prologue(args):
 
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     sampler.start()
-    warm = 0
+    # exactly the requested warm-up steps, then untimed launches (reported apart) until the
+    # clock sampler has run for a second
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    settle = 0
     t_w = time.perf_counter()
     with torch.cuda.stream(stream):
-        while warm < max(3, args.warmup) or time.perf_counter() - t_w < 1.0:
+        while time.perf_counter() - t_w < 1.0:
             step()
-            warm += 1
+            settle += 1
+            if settle % 16 == 0:
+                stream.synchronize()
     stream.synchronize()
     if args.steps is None:
         w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -529,7 +537,11 @@ def run_prologue(args):
         in_bytes = 3 * w.T * w.H * w.D * 2 + 2 * w.T * w.D * 4 + (8 * w.D if w.qk_norm else 0)
         result = {
             "metric": metric, "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
-            "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "clock_settle_launches": {
+                "launches": settle,
+                "why": "untimed launches after the warm-up, until the nvidia-smi clock sampler (200 ms period) "
+                       "has run for 1 s, so that the clocks line reflects the GPU under load"},
             "vs_baseline": None, "dtype": synth.DTYPE_NAMES[w.dtype],
             "data": "synthetic (seeded normals; 2-D rope tables of the patch grid)",
             "config": {"workload": w.name, "images": w.images, "grid": list(w.grid), "tokens": w.T, "H": w.H,
@@ -633,13 +645,22 @@ def main():
 
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
     sampler.start()
-    t_w = time.perf_counter()
-    warm_done = 0
+    # exactly the requested warm-up steps, then (untimed, reported apart) more launches until the
+    # clock sampler has run for a second: nvidia-smi samples every 200 ms, and a short timed
+    # region alone would hold too few samples to show the clocks under load
     with torch.cuda.stream(stream):
-        while warm_done < args.warmup or time.perf_counter() - t_w < 1.0:
+        for i in range(args.warmup):
             step()
-            warm_done += 1
-            if warm_done % 16 == 0:
+            if (i + 1) % 16 == 0:
+                stream.synchronize()
+    stream.synchronize()
+    t_w = time.perf_counter()
+    settle_done = 0
+    with torch.cuda.stream(stream):
+        while time.perf_counter() - t_w < 1.0:
+            step()
+            settle_done += 1
+            if settle_done % 16 == 0:
                 stream.synchronize()
     stream.synchronize()
     if args.steps is None:
@@ -739,7 +760,11 @@ def main():
             "unit": "TFLOP/s",
             "n_gpus": world,
             "steps": args.steps,
-            "warmup": warm_done,
+            "warmup": args.warmup,
+            "clock_settle_launches": {
+                "launches": settle_done,
+                "why": "untimed launches after the warm-up, until the nvidia-smi clock sampler (200 ms period) "
+                       "has run for 1 s, so that the clocks line reflects the GPU under load"},
             "ms_per_step": ms_step,
             "higher_is_better": True,
             "scaling": "weak",
@@ -763,6 +788,7 @@ def main():
                 "peak": peak,
                 "unit": "TFLOP/s",
                 "frac": per_gpu_tflops / peak,
+                "frac_of_datasheet": per_gpu_tflops / DATASHEET_PEAK_TFLOPS,
                 "traffic": traffic,
                 "peak_source": peak_note if peaks else "fallback",
                 "kernel": "vitattn::fwd_kernel",
