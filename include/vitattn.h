@@ -25,7 +25,9 @@
  *   vitattn_forward_ext      Lq != Lk, aligned causal mask, log-sum-exp output
  *   vitattn_qkv_rope         the prologue: packed QKV split + rotary embedding
  *   vitattn_qkv_norm_rope    the same with a per-head q/k RMS norm before the rope
- *   vitattn_forward_host     vitattn_forward from host buffers (copies enqueued)
+ *   vitattn_forward_strided  vitattn_forward on token-strided inputs (a packed projection)
+ *   vitattn_qk_rope, vitattn_qk_norm_rope  the prologues without the v copy
+ *   vitattn_forward_host     vitattn_forward from host buffers (copies overlapped)
  *   ..._checked, ..._check_args*, vitattn_strerror, vitattn_last_cuda_error,
  *   vitattn_version, vitattn_launches_per_call: synchronising variants for
  *   tests, argument checks alone, status text, versioning.
@@ -56,8 +58,17 @@
  * wait that runs out ends the kernel early and records VITATTN_ERR_TIMEOUT in
  * a device status word, which vitattn_forward_checked reports.
  *
+ * Devices.  Every call runs on the current CUDA device.  Each device pointer
+ * must be that device's memory (or managed / mapped pinned memory); a
+ * pointer to plain host memory or to another GPU's memory is refused with
+ * VITATTN_ERR_DEVICE before anything is enqueued.
+ *
  * Thread safety.  Calls may come from several host threads; each call
- * launches on its own stream argument.
+ * launches on its own stream argument and keeps no state between calls.
+ * One exception: the ..._checked entries (meant for tests) read two status
+ * words that every call of the library on a device shares, so checked calls
+ * that overlap in time on one device (several threads or streams) can see
+ * each other's timeout or range report.
  */
 #ifndef VITATTN_H
 #define VITATTN_H
@@ -95,7 +106,8 @@ enum vitattn_status {
     VITATTN_ERR_CUDA = -7,    /* the CUDA runtime or driver returned an error */
     VITATTN_ERR_TIMEOUT = -8, /* a bounded in-kernel wait ran out (checked entry only) */
     VITATTN_ERR_SCALE = -9,   /* scale is NaN or infinite (or eps negative / not finite) */
-    VITATTN_ERR_DEVICE = -10, /* the current device is not an sm_100 GPU */
+    VITATTN_ERR_DEVICE = -10, /* the current device is not an sm_100 GPU, or a pointer argument is plain
+                                 host memory or another GPU's memory */
     VITATTN_ERR_RANGE = -11,  /* a bf16 V value has |v| >= 65536 (checked entry only) */
     VITATTN_ERR_SEQLENS = -12 /* cu_seqlens does not start at 0 or decreases somewhere */
 };
@@ -292,17 +304,89 @@ VITATTN_API int vitattn_check_args_qkv_norm_rope(const void* qkv, const float* c
                                                  int64_t H, int64_t D, int dtype);
 
 /*
- * vitattn_forward_host -- the same operation from HOST buffers: enqueues the
- * copies hq->dq, hk->dk, hv->dv, the kernel, and dout->hout, in that order,
- * on `stream`, and returns without synchronising.  Source: hanzo-ml
+ * vitattn_forward_strided -- vitattn_forward on inputs whose tokens are not
+ * packed back to back: element (b, i, h, d) of q sits at
+ * q[((b*N + i)*q_stride + h*D + d)], likewise k (k_stride) and v (v_stride).
+ * The use: a QKV linear writes one packed [B, N, 3, H, D] projection; with
+ * q = qkv, k = qkv + H*D, v = qkv + 2*H*D and all strides 3*H*D the attention
+ * reads it in place, and after vitattn_qk_rope (which rotates q and k into
+ * their own buffers) v still comes straight from the projection, so the
+ * prologue never copies it.  Source: inferencelayer "src/vision_gpu.rs",
+ * VIS_QKV_ROPE doc (the projection output is q | k | v per token; the
+ * attention's q, k, v are three column ranges of it).
+ *   q_stride, k_stride, v_stride  elements between consecutive tokens,
+ *             each >= H*D and a multiple of 8 (token rows start on 16 bytes);
+ *             H*D everywhere is exactly vitattn_forward.
+ *   out       dense [B, N, H, D], not overlapping any input's span; the
+ *             inputs may overlap one another (views of one projection).
+ *   Everything else as for vitattn_forward (VITATTN_ERR_DIM for a bad stride).
+ */
+VITATTN_API int vitattn_forward_strided(const void* q, const void* k, const void* v, void* out, int64_t B,
+                                        int64_t N, int64_t H, int64_t D, int64_t q_stride, int64_t k_stride,
+                                        int64_t v_stride, float scale, int dtype, vitattn_stream_t stream);
+
+/* vitattn_forward_strided, then a stream synchronisation and a read of the kernel's status words. */
+VITATTN_API int vitattn_forward_strided_checked(const void* q, const void* k, const void* v, void* out, int64_t B,
+                                                int64_t N, int64_t H, int64_t D, int64_t q_stride,
+                                                int64_t k_stride, int64_t v_stride, float scale, int dtype,
+                                                vitattn_stream_t stream);
+
+/* The argument checks of vitattn_forward_strided alone (no CUDA call). */
+VITATTN_API int vitattn_check_args_strided(const void* q, const void* k, const void* v, const void* out, int64_t B,
+                                           int64_t N, int64_t H, int64_t D, int64_t q_stride, int64_t k_stride,
+                                           int64_t v_stride, float scale, int dtype);
+
+/*
+ * vitattn_qk_rope -- vitattn_qkv_rope without the v output: q and k are
+ * rotated into [T, H, D] buffers and v is neither read nor written (the
+ * attention reads it from qkv through vitattn_forward_strided with
+ * v_stride = 3*H*D).  Source: inferencelayer "src/vision_gpu.rs",
+ * VIS_QKV_ROPE and its doc ("pure data movement plus one rotation": the
+ * rotation applies to q and k only).  Arguments and errors as for
+ * vitattn_qkv_rope without v.  Enqueues one kernel on `stream`.
+ */
+VITATTN_API int vitattn_qk_rope(const void* qkv, const float* cos_table, const float* sin_table, void* q, void* k,
+                                int64_t T, int64_t H, int64_t D, int dtype, vitattn_stream_t stream);
+
+/* The argument checks of vitattn_qk_rope alone (no CUDA call). */
+VITATTN_API int vitattn_check_args_qk_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                                           const void* q, const void* k, int64_t T, int64_t H, int64_t D,
+                                           int dtype);
+
+/*
+ * vitattn_qk_norm_rope -- vitattn_qkv_norm_rope without the v output (v
+ * stays in qkv, as for vitattn_qk_rope).  Source: inferencelayer
+ * "src/vision_gpu.rs", GLM_QKV_QKNORM_ROPE and its doc.
+ */
+VITATTN_API int vitattn_qk_norm_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                                     const float* q_norm_w, const float* k_norm_w, float eps, void* q, void* k,
+                                     int64_t T, int64_t H, int64_t D, int dtype, vitattn_stream_t stream);
+
+/* The argument checks of vitattn_qk_norm_rope alone (no CUDA call). */
+VITATTN_API int vitattn_check_args_qk_norm_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                                                const float* q_norm_w, const float* k_norm_w, float eps,
+                                                const void* q, const void* k, int64_t T, int64_t H, int64_t D,
+                                                int dtype);
+
+/*
+ * vitattn_forward_host -- the same operation from HOST buffers: the copies
+ * hq->dq, hk->dk, hv->dv, the attention, and dout->hout.  Source: hanzo-ml
  * "src/vulkan_backend.rs", `flash_attn` (the host-data convenience form of
  * `flash_attn_gpu`: upload the inputs, run the device entry, read the
  * output back).  Here the caller supplies the device staging buffers, so
- * the library still allocates nothing.  The caller synchronises
- * the stream before reading hout.  Host buffers should be pinned
- * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous; the
- * device buffers dq, dk, dv, dout are caller-owned staging with the same
- * requirements as in vitattn_forward.  All eight pointers are required.
+ * the library still allocates no memory.
+ *   The batch is split into up to 8 groups of whole images; group c's
+ *   inputs are copied in while the kernel of group c-1 runs and the output
+ *   of group c-2 is copied out.  The copies run on two streams the library
+ *   keeps per host thread and device (created on the first call); the
+ *   kernels run on `stream`.  The copies start after the work already
+ *   enqueued on `stream`, and work enqueued on `stream` after this call (or
+ *   a synchronisation of `stream`) comes after the last output copy, so the
+ *   caller synchronises `stream` before reading hout, as with one stream.
+ *   Host buffers should be pinned (cudaHostAlloc / cudaHostRegister) for the
+ *   copies to overlap; dq, dk, dv, dout are caller-owned device staging with
+ *   the requirements of vitattn_forward.  All eight pointers are required.
+ *   Launches one kernel per group.
  */
 VITATTN_API int vitattn_forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq,
                          void* dk, void* dv, void* dout, int64_t B, int64_t N, int64_t H,

@@ -258,7 +258,8 @@ def test_every_compute_entry_cites_the_passage_that_defines_it():
     to the page (by source path) that defines it."""
     text = open(HEADER).read()
     compute = {"vitattn_forward", "vitattn_forward_ext", "vitattn_forward_gqa", "vitattn_forward_varlen",
-               "vitattn_qkv_rope", "vitattn_qkv_norm_rope", "vitattn_forward_host"}
+               "vitattn_qkv_rope", "vitattn_qkv_norm_rope", "vitattn_forward_host", "vitattn_forward_strided",
+               "vitattn_qk_rope", "vitattn_qk_norm_rope"}
     seen = set()
     for m in re.finditer(r"/\*(.*?)\*/\s*VITATTN_API[^;(]*?\b(vitattn_\w+)\s*\(", text, re.S):
         comment, name = m.group(1), m.group(2)
@@ -266,3 +267,48 @@ def test_every_compute_entry_cites_the_passage_that_defines_it():
             assert re.search(r"src/[\w/]+\.rs", comment), f"{name}: no source citation"
             seen.add(name)
     assert seen == compute
+
+
+# ------------------------------------------------------------------ token-strided inputs
+
+def check_strided(**kw):
+    B, N, H, D = kw.get("B", 2), kw.get("N", 100), 2, 64
+    row = H * D
+    ts = kw.get("ts", 3 * row)
+    span = ((B * N - 1) * ts + row) * 2  # bytes one strided input reaches
+    qkv = A
+    a = dict(q=qkv, k=qkv + 2 * row, v=qkv + 4 * row, out=A + span + 4 * row + 64, B=B, N=N, H=H, D=D,
+             tq=ts, tk=ts, tv=ts, scale=0.125, dtype=vitattn.BF16)
+    a.update(kw)
+    return vitattn.check_args_strided(a["q"], a["k"], a["v"], a["out"], a["B"], a["N"], a["H"], a["D"], a["tq"],
+                                      a["tk"], a["tv"], a["scale"], a["dtype"])
+
+
+def test_strided_views_of_one_projection_pass():
+    # q, k, v as the three column ranges of one packed [B, N, 3, H, D] projection
+    assert check_strided() == 0
+    # dense strides are the plain layout
+    assert check_strided(ts=128, tq=128, tk=128, tv=128, k=A + 2 * 100 * 256 * 2, v=A + 4 * 100 * 256 * 2,
+                         out=A + 6 * 100 * 256 * 2) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), -1), (dict(v=0), -1), (dict(tq=64), -2), (dict(tk=132), -2), (dict(tv=0), -2), (dict(B=0), -2),
+    (dict(D=60), -3), (dict(dtype=5), -4), (dict(k=A + 2 * 128 + 8), -5), (dict(out=A + 96), -6),
+    (dict(out=A + ((2 * 100 - 1) * 384 + 128) * 2 + 2 * 128 - 16), -6), (dict(scale=float("nan")), -9),
+])
+def test_strided_argument_errors(kw, code):
+    assert check_strided(**kw) == code
+
+
+def test_qk_rope_checks_need_no_v_and_refuse_aliasing():
+    T, H, D = 16, 2, 64
+    qkv = A
+    inb = T * 3 * H * D * 2
+    cs, sn = A + inb, A + inb + T * D * 4
+    q, k = sn + T * D * 4, sn + T * D * 4 + T * H * D * 2
+    assert vitattn.check_args_qk_rope(qkv, cs, sn, q, k, T, H, D, vitattn.BF16) == 0
+    assert vitattn.check_args_qk_rope(qkv, cs, sn, q, q, T, H, D, vitattn.BF16) == -6   # q and k overlap
+    assert vitattn.check_args_qk_rope(qkv, cs, sn, qkv + 64, k, T, H, D, vitattn.BF16) == -6  # q inside qkv
+    assert vitattn.check_args_qk_rope(qkv, cs, sn, 0, k, T, H, D, vitattn.BF16) == -1
+    assert vitattn.check_args_qk_rope(qkv, cs, sn, q, k, T, H, 72, 7) == -4

@@ -89,3 +89,24 @@ def test_unsupported_dtype_is_a_type_error():
 def test_status_errors_carry_their_code_and_text():
     e = vitattn.VitAttnError(-9, "vitattn_qkv_norm_rope")
     assert e.status == -9 and "vitattn_qkv_norm_rope" in str(e) and "finite" in str(e)
+
+
+def test_tensors_on_different_devices_are_refused():
+    # every wrapper calls this check after its shape checks and before the
+    # library; a tensor on another device than the first one raises
+    a = torch.zeros(4)
+    b = torch.zeros(4, device="meta")
+    vitattn._same_device("t", a, a.clone(), a.clone())
+    with pytest.raises(ValueError, match="device"):
+        vitattn._same_device("t", a, a.clone(), b)
+
+
+def test_a_stream_of_another_device_is_refused():
+    class FakeStream:
+        device = torch.device("cuda", 1)
+        cuda_stream = 1234
+
+    assert vitattn._stream_handle(77, torch.device("cuda", 0)) == 77
+    assert vitattn._stream_handle(FakeStream(), torch.device("cuda", 1)) == 1234
+    with pytest.raises(ValueError, match="stream"):
+        vitattn._stream_handle(FakeStream(), torch.device("cuda", 0))

@@ -266,6 +266,44 @@ def test_host_buffer_entry_matches(cuda_device):
     assert_close(got, oracle.attention(q, k, v, w.scale, w.dtype))
 
 
+@pytest.mark.parametrize("B", [9, 16])
+def test_host_buffer_entry_multi_group(cuda_device, B):
+    # the batch travels in groups of whole images (up to 8 groups, the last one
+    # shorter when B does not divide); every image's output must match the oracle,
+    # and a second call on the same buffers gives the same bits
+    import torch
+
+    q, k, v = synth.random_qkv(B, 200, 4, 64, synth.BF16, seed=31 + B)
+    hosts = [torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).pin_memory() for x in (q, k, v)]
+    hout = torch.full_like(hosts[0], float("nan")).pin_memory()
+    dq, dk, dv, dout = (torch.empty(q.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    s = torch.cuda.Stream()
+    args = [h.data_ptr() for h in hosts] + [hout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                            dout.data_ptr(), B, 200, 4, 64, 0.125, synth.BF16, s.cuda_stream]
+    assert vitattn.forward_host_ptr(*args) == 0
+    s.synchronize()
+    first = from_dev(hout, synth.BF16)
+    assert_close(first, oracle.attention(q, k, v, 0.125, synth.BF16), f"B={B}")
+    hout.fill_(float("nan"))
+    assert vitattn.forward_host_ptr(*args) == 0
+    s.synchronize()
+    assert np.array_equal(from_dev(hout, synth.BF16), first)
+
+
+def test_pointers_of_host_memory_are_refused(cuda_device):
+    # a plain (unregistered) host pointer passed as device memory is refused
+    # before anything is enqueued, instead of reaching a tensor map
+    import torch
+
+    t = torch.zeros((1, 64, 2, 64), dtype=torch.bfloat16, device="cuda")
+    o = torch.zeros_like(t)
+    h = np.zeros(64 * 2 * 64 + 8, dtype=np.uint16)
+    hp = (h.ctypes.data + 15) // 16 * 16
+    assert vitattn.forward_ptr(hp, t.data_ptr(), t.data_ptr(), o.data_ptr(), 1, 64, 2, 64, 1.0, 0) == -10
+    assert vitattn.forward_ptr(t.data_ptr(), t.data_ptr(), t.data_ptr(), hp, 1, 64, 2, 64, 1.0, 0) == -10
+    torch.cuda.synchronize()
+
+
 def test_errors_on_device_do_not_launch(cuda_device):
     import torch
 

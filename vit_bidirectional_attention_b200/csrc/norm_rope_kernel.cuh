@@ -6,7 +6,8 @@
 // head's q row x (and k row) is first normalised over its D elements,
 //     y[d] = x[d] / sqrt(mean_e x[e]^2 + eps) * w[d],
 // with one weight vector w[D] for q and another for k, shared by all heads;
-// the rotation is then applied to y (norm first, rope second).  v is copied.
+// the rotation is then applied to y (norm first, rope second).  v is copied
+// (kCopyV), or left in the packed projection for the attention to read there.
 //
 // Same thread layout as qkv_rope_kernel: one warp per (token, head), lane l
 // holding elements 4l..4l+3.  Since the norm is one factor per head row,
@@ -51,7 +52,7 @@ __device__ __forceinline__ uint2 norm_rotate4(uint2 x, uint2 p, float inv, float
 // Resident blocks per SM (the grid is this many per SM).
 constexpr int kNormRopeBlocksPerSm = 3;
 
-template <bool kBF16>
+template <bool kBF16, bool kCopyV>
 __global__ void __launch_bounds__(kRopeThreads, kNormRopeBlocksPerSm) qkv_norm_rope_kernel(
     const uint8_t* __restrict__ qkv, const float* __restrict__ cs, const float* __restrict__ sn,
     const float* __restrict__ qw, const float* __restrict__ kw, float eps, uint8_t* __restrict__ q,
@@ -86,7 +87,7 @@ __global__ void __launch_bounds__(kRopeThreads, kNormRopeBlocksPerSm) qkv_norm_r
                 const uint8_t* src = qkv + in0 + (size_t)r * head2;
                 xq[r] = ld_nc_v2(src);
                 xk[r] = ld_nc_v2(src + hd2);
-                xv[r] = ld_nc_v2(src + 2u * hd2);
+                if (kCopyV) xv[r] = ld_nc_v2(src + 2u * hd2);
             }
         }
         float4 Aq = make_float4(0.f, 0.f, 0.f, 0.f), Bq = Aq, Ak = Aq, Bk = Aq;
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(kRopeThreads, kNormRopeBlocksPerSm) qkv_norm_r
                 const size_t o = out0 + (size_t)r * head2;
                 st_v2(q + o, norm_rotate4<kBF16>(xq[r], pq, iq, Aq, Bq));
                 st_v2(k + o, norm_rotate4<kBF16>(xk[r], pk, ik, Ak, Bk));
-                st_v2(v + o, xv[r]);
+                if (kCopyV) st_v2(v + o, xv[r]);
             }
         }
     }

@@ -9,7 +9,9 @@
 //     x'[d] = x[d] * cos[d] + rotate_half(x)[d] * sin[d],
 //     rotate_half(x)[d] = -x[d + D/2] (d < D/2),  x[d - D/2] (d >= D/2),
 // for q and k; v is copied.  Outputs are token-major [T, H, D], the layout
-// the attention kernel reads.
+// the attention kernel reads.  With kCopyV = false v is neither read nor
+// written: the attention then reads it straight out of the packed
+// projection (token stride 3*H*D), and the prologue moves a third fewer bytes.
 //
 // The pass is pure HBM traffic (read 3*T*H*D elements and the tables, write
 // 3*T*H*D elements), so the design is about coalescing: one warp per (token,
@@ -79,7 +81,7 @@ __device__ __forceinline__ uint2 rotate4(uint2 x, uint2 p, float4 c, float4 s, f
 // token's cos/sin row is loaded once for all of them.
 constexpr int kRopeHeadsPerWarp = 4;
 
-template <bool kBF16>
+template <bool kBF16, bool kCopyV>
 __global__ void __launch_bounds__(kRopeThreads, 4) qkv_rope_kernel(const uint8_t* __restrict__ qkv,
                                                                    const float* __restrict__ cs,
                                                                    const float* __restrict__ sn,
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(kRopeThreads, 4) qkv_rope_kernel(const uint8_t
                 const uint8_t* src = qkv + in0 + (size_t)r * head2;
                 xq[r] = ld_nc_v2(src);
                 xk[r] = ld_nc_v2(src + hd2);
-                xv[r] = ld_nc_v2(src + 2u * hd2);
+                if (kCopyV) xv[r] = ld_nc_v2(src + 2u * hd2);
             }
         }
 #pragma unroll
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kRopeThreads, 4) qkv_rope_kernel(const uint8_t
                 const size_t o = out0 + (size_t)r * head2;
                 st_v2(q + o, rotate4<kBF16>(xq[r], pq, c, s, sign));
                 st_v2(k + o, rotate4<kBF16>(xk[r], pk, c, s, sign));
-                st_v2(v + o, xv[r]);
+                if (kCopyV) st_v2(v + o, xv[r]);
             }
         }
     }

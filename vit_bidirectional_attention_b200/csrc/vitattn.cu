@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 
 #include "vitattn.h"
@@ -110,6 +111,42 @@ int check_args_gqa(const void* q, const void* k, const void* v, const void* out,
     return VITATTN_OK;
 }
 
+// Token-strided inputs: element (b, i, h, d) of x at x + ((b*N + i)*ts_x + h*D + d)
+// for x = q, k, v (ts_x elements between consecutive tokens, >= H*D, a multiple
+// of 8 so that every token row starts on 16 bytes); out dense [B, N, H, D].
+// The inputs may overlap one another (views of one packed projection); out
+// must not overlap any of them.
+int check_args_strided(const void* q, const void* k, const void* v, const void* out, int64_t B, int64_t N,
+                       int64_t H, int64_t D, const int64_t ts[3], float scale, int dtype) {
+    if (!q || !k || !v || !out) return VITATTN_ERR_NULL;
+    if (B < 1 || N < 1 || H < 1 || D < 1) return VITATTN_ERR_DIM;
+    if (D < 16 || D > 128 || D % 8 != 0) return VITATTN_ERR_HEADDIM;
+    if (dtype != VITATTN_BF16 && dtype != VITATTN_F16) return VITATTN_ERR_DTYPE;
+    if (!std::isfinite(scale)) return VITATTN_ERR_SCALE;
+    if (N > (int64_t)INT32_MAX - 512 || H > (int64_t)INT32_MAX || B > (int64_t)INT32_MAX) return VITATTN_ERR_DIM;
+    const uint64_t row = (uint64_t)H * (uint64_t)D;  // elements of one token's heads
+    if (row * 2u >= (1ull << 40)) return VITATTN_ERR_DIM;
+    const uint64_t out_bytes_batch = (uint64_t)N * row * 2u;
+    if (out_bytes_batch >= (1ull << 40) || (uint64_t)B > (1ull << 62) / out_bytes_batch) return VITATTN_ERR_DIM;
+    const uint64_t work = (uint64_t)B * (uint64_t)H * (uint64_t)((N + 255) / 256);
+    if (work > (uint64_t)INT32_MAX) return VITATTN_ERR_DIM;
+    uint64_t extent[3];
+    for (int i = 0; i < 3; ++i) {
+        if (ts[i] < (int64_t)row || ts[i] % 8 != 0) return VITATTN_ERR_DIM;
+        const uint64_t batch = (uint64_t)N * (uint64_t)ts[i] * 2u;  // bytes between batches (a TMA stride)
+        if (batch >= (1ull << 40) || (uint64_t)B > (1ull << 62) / batch) return VITATTN_ERR_DIM;
+        extent[i] = ((uint64_t)B * (uint64_t)N - 1u) * (uint64_t)ts[i] * 2u + row * 2u;
+    }
+    const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                           reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out)) & 15u;
+    if (mis) return VITATTN_ERR_ALIGN;
+    const uint64_t out_bytes = out_bytes_batch * (uint64_t)B;
+    if (overlaps2(out, out_bytes, q, extent[0]) || overlaps2(out, out_bytes, k, extent[1]) ||
+        overlaps2(out, out_bytes, v, extent[2]))
+        return VITATTN_ERR_ALIAS;
+    return VITATTN_OK;
+}
+
 // Ragged batch: q, k, v, out are [total, H, D] with total = cu_seqlens[num_seqs];
 // cu_seqlens (host) starts at 0 and never decreases.
 int check_args_varlen(const void* q, const void* k, const void* v, const void* out,
@@ -142,9 +179,11 @@ int check_args_varlen(const void* q, const void* k, const void* v, const void* o
 }
 
 // QKV split + rope prologue: qkv [T, 3, H, D], cos/sin [T, D] f32, q/k/v [T, H, D].
+// need_v = false: the q/k-only prologue (v stays in qkv), v is not an output.
 int check_args_rope(const void* qkv, const float* cs, const float* sn, const void* q, const void* k,
-                    const void* v, int64_t T, int64_t H, int64_t D, int dtype) {
-    if (!qkv || !cs || !sn || !q || !k || !v) return VITATTN_ERR_NULL;
+                    const void* v, int64_t T, int64_t H, int64_t D, int dtype, bool need_v = true) {
+    if (!qkv || !cs || !sn || !q || !k || (need_v && !v)) return VITATTN_ERR_NULL;
+    if (!need_v) v = q;  // stands in for the absent output in the checks below
     if (T < 1 || H < 1 || D < 1) return VITATTN_ERR_DIM;
     if (D < 16 || D > 128 || D % 8 != 0) return VITATTN_ERR_HEADDIM;
     if (dtype != VITATTN_BF16 && dtype != VITATTN_F16) return VITATTN_ERR_DTYPE;
@@ -158,7 +197,8 @@ int check_args_rope(const void* qkv, const float* cs, const float* sn, const voi
     const uint64_t in_bytes = 3u * row_bytes * (uint64_t)T, out_bytes = row_bytes * (uint64_t)T;
     const uint64_t tab_bytes = (uint64_t)T * (uint64_t)D * 4u;
     const void* outs[3] = {q, k, v};
-    for (int i = 0; i < 3; ++i) {
+    const int nout = need_v ? 3 : 2;
+    for (int i = 0; i < nout; ++i) {
         if (overlaps2(outs[i], out_bytes, qkv, in_bytes) || overlaps2(outs[i], out_bytes, cs, tab_bytes) ||
             overlaps2(outs[i], out_bytes, sn, tab_bytes))
             return VITATTN_ERR_ALIAS;
@@ -172,9 +212,10 @@ int check_args_rope(const void* qkv, const float* cs, const float* sn, const voi
 // vectors (16-byte aligned, not overlapping an output) and a finite eps >= 0.
 int check_args_norm_rope(const void* qkv, const float* cs, const float* sn, const float* qw, const float* kw,
                          float eps, const void* q, const void* k, const void* v, int64_t T, int64_t H,
-                         int64_t D, int dtype) {
-    int rc = check_args_rope(qkv, cs, sn, q, k, v, T, H, D, dtype);
+                         int64_t D, int dtype, bool need_v = true) {
+    int rc = check_args_rope(qkv, cs, sn, q, k, v, T, H, D, dtype, need_v);
     if (rc) return rc;
+    if (!need_v) v = q;
     if (!qw || !kw) return VITATTN_ERR_NULL;
     if ((reinterpret_cast<uintptr_t>(qw) | reinterpret_cast<uintptr_t>(kw)) & 15u) return VITATTN_ERR_ALIGN;
     if (!std::isfinite(eps) || eps < 0.f) return VITATTN_ERR_SCALE;
@@ -204,13 +245,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Token-major [B, N, H, D] seen by TMA as 4-D {D, H, N, B} (innermost first);
 // one box is `width` head-dim columns x 1 head x 128 tokens x 1 batch.
+// `ts` is the element stride between consecutive tokens (H*D when dense).
 bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t N, int64_t H,
-                int64_t D, int width) {
+                int64_t D, int width, int64_t ts) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)(D * 2), (cuuint64_t)(H * D * 2),
-                                   (cuuint64_t)(N * H * D * 2)};
+    const cuuint64_t strides[3] = {(cuuint64_t)(D * 2), (cuuint64_t)(ts * 2), (cuuint64_t)(N * ts * 2)};
     const cuuint32_t box[4] = {(cuuint32_t)width, 1u, (cuuint32_t)vitattn::kTileRows, 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     const CUtensorMapSwizzle sw = width == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -294,6 +335,30 @@ int device_info(int* num_sms) {
     return VITATTN_OK;
 }
 
+// Every pointer must address memory that the current device's kernels may
+// read and write: its own device memory, managed memory, or pinned host
+// memory mapped for it.  Plain (unregistered) host memory or another GPU's
+// memory would be encoded into a tensor map and fault or be read across
+// devices, so the call is refused before anything is enqueued.
+int check_device_ptrs(std::initializer_list<const void*> ptrs) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    for (const void* ptr : ptrs) {
+        if (!ptr) continue;
+        cudaPointerAttributes a;
+        e = cudaPointerGetAttributes(&a, ptr);
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();  // clear the sticky-free error of the query
+            return VITATTN_ERR_DEVICE;
+        }
+        if (a.type == cudaMemoryTypeUnregistered) return VITATTN_ERR_DEVICE;
+        if (a.type == cudaMemoryTypeDevice && a.device != dev) return VITATTN_ERR_DEVICE;
+        if (a.type == cudaMemoryTypeHost && a.devicePointer == nullptr) return VITATTN_ERR_DEVICE;
+    }
+    return VITATTN_OK;
+}
+
 // The dynamic shared-memory limit of one kernel instantiation, raised once per device.
 int ensure_smem(int dp, int dtype, Mode mode, const void* fn) {
     int dev = 0;
@@ -311,9 +376,10 @@ int ensure_smem(int dp, int dtype, Mode mode, const void* fn) {
 }
 
 // Tensor maps of q, k, v for every column-chunk width, and the shape fields.
+// ts: token strides of q, k, v in elements (nullptr: dense, heads * D).
 int fill_common(FwdParams* prm, const void* q, const void* k, const void* v, void* out, int64_t B,
                 int64_t N, int64_t H, int64_t D, float scale, int dtype, int flags, int64_t Hkv = 0,
-                int64_t Nk = 0) {
+                int64_t Nk = 0, const int64_t* ts = nullptr) {
     std::memset(prm, 0, sizeof *prm);
     if (Hkv == 0) Hkv = H;  // multi-head: k and v have the query's head count
     if (Nk == 0) Nk = N;    // self-attention: as many keys as queries
@@ -326,7 +392,9 @@ int fill_common(FwdParams* prm, const void* q, const void* k, const void* v, voi
         const int w = vitattn::chunk_width(dp, c);
         for (int m = 0; m < 3; ++m) {
             CUtensorMap* map = &prm->maps[m][vitattn::width_class(w)];
-            if (!encode_map(map, src[m], dtype, B, lens[m], heads[m], D, w)) return cuda_fail(cudaErrorInvalidValue);
+            const int64_t stride = ts ? ts[m] : heads[m] * D;
+            if (!encode_map(map, src[m], dtype, B, lens[m], heads[m], D, w, stride))
+                return cuda_fail(cudaErrorInvalidValue);
         }
     }
     prm->kv_group = (int)(H / Hkv);
@@ -361,23 +429,27 @@ struct Ext {
     int64_t Nk = 0;       // keys per (b, h); 0: N
     int causal = 0;       // aligned causal mask
     float* lse = nullptr; // optional [B, H, N] log-sum-exp output
+    const int64_t* ts = nullptr;  // token strides of q, k, v in elements; nullptr: dense
 };
 
 int launch(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
            int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags, int64_t Hkv = 0,
            const Ext& ext = Ext()) {
-    int rc = ext.Nk ? check_args_ext(q, k, v, out, ext.lse, B, N, ext.Nk, H, D, scale, dtype)
-             : Hkv  ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
-                    : check_args(q, k, v, out, B, N, H, D, scale, dtype);
+    int rc = ext.ts   ? check_args_strided(q, k, v, out, B, N, H, D, ext.ts, scale, dtype)
+             : ext.Nk ? check_args_ext(q, k, v, out, ext.lse, B, N, ext.Nk, H, D, scale, dtype)
+             : Hkv    ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
+                      : check_args(q, k, v, out, B, N, H, D, scale, dtype);
     if (rc) return rc;
     const int64_t Nk = ext.Nk ? ext.Nk : N;
     const int dp = (int)((D + 15) / 16 * 16);
     int num_sms = 0;
     rc = device_info(&num_sms);
     if (rc) return rc;
+    rc = check_device_ptrs({q, k, v, out, ext.lse});
+    if (rc) return rc;
 
     FwdParams prm;
-    rc = fill_common(&prm, q, k, v, out, B, N, H, D, scale, dtype, flags, Hkv, Nk);
+    rc = fill_common(&prm, q, k, v, out, B, N, H, D, scale, dtype, flags, Hkv, Nk, ext.ts);
     if (rc) return rc;
     prm.causal = ext.causal ? 1 : 0;
     prm.causal_off = (int)(Nk - N);
@@ -420,6 +492,8 @@ int launch_varlen(const void* q, const void* k, const void* v, void* out, const 
     int num_sms = 0;
     rc = device_info(&num_sms);
     if (rc) return rc;
+    rc = check_device_ptrs({q, k, v, out});
+    if (rc) return rc;
 
     FwdParams prm;
     rc = fill_common(&prm, q, k, v, out, 1, total, H, D, scale, dtype, flags);
@@ -450,11 +524,13 @@ int launch_varlen(const void* q, const void* k, const void* v, void* out, const 
 // The prologue: a grid-stride kernel, 8 warps per block, at most 8 blocks per SM
 // (a full SM), one warp per (token, head).
 int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void* k, void* v, int64_t T,
-                int64_t H, int64_t D, int dtype, cudaStream_t stream) {
-    int rc = check_args_rope(qkv, cs, sn, q, k, v, T, H, D, dtype);
+                int64_t H, int64_t D, int dtype, cudaStream_t stream, bool copy_v = true) {
+    int rc = check_args_rope(qkv, cs, sn, q, k, v, T, H, D, dtype, copy_v);
     if (rc) return rc;
     int num_sms = 0;
     rc = device_info(&num_sms);
+    if (rc) return rc;
+    rc = check_device_ptrs({qkv, cs, sn, q, k, copy_v ? v : nullptr});
     if (rc) return rc;
     const uint64_t items = (uint64_t)T * (uint64_t)((H + vitattn::kRopeHeadsPerWarp - 1) / vitattn::kRopeHeadsPerWarp);
     const uint64_t per_block = (uint64_t)(vitattn::kRopeThreads / 32);
@@ -465,8 +541,11 @@ int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void
     long long TT = (long long)T;
     int HH = (int)H, DD = (int)D;
     void* args[9] = {&qkv8, &cs, &sn, &q8, &k8, &v8, &TT, &HH, &DD};
-    const void* fn = dtype == VITATTN_BF16 ? reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true>)
-                                           : reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false>);
+    const bool bf = dtype == VITATTN_BF16;
+    const void* fn = copy_v ? (bf ? reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true, true>)
+                                  : reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false, true>))
+                            : (bf ? reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true, false>)
+                                  : reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false, false>));
     cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(vitattn::kRopeThreads), args, 0, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return VITATTN_OK;
@@ -476,11 +555,13 @@ int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void
 // that are resident at once (kNormRopeBlocksPerSm per SM).
 int launch_norm_rope(const void* qkv, const float* cs, const float* sn, const float* qw, const float* kw,
                      float eps, void* q, void* k, void* v, int64_t T, int64_t H, int64_t D, int dtype,
-                     cudaStream_t stream) {
-    int rc = check_args_norm_rope(qkv, cs, sn, qw, kw, eps, q, k, v, T, H, D, dtype);
+                     cudaStream_t stream, bool copy_v = true) {
+    int rc = check_args_norm_rope(qkv, cs, sn, qw, kw, eps, q, k, v, T, H, D, dtype, copy_v);
     if (rc) return rc;
     int num_sms = 0;
     rc = device_info(&num_sms);
+    if (rc) return rc;
+    rc = check_device_ptrs({qkv, cs, sn, qw, kw, q, k, copy_v ? v : nullptr});
     if (rc) return rc;
     const uint64_t items = (uint64_t)T * (uint64_t)((H + vitattn::kRopeHeadsPerWarp - 1) / vitattn::kRopeHeadsPerWarp);
     const uint64_t per_block = (uint64_t)(vitattn::kRopeThreads / 32);
@@ -492,8 +573,12 @@ int launch_norm_rope(const void* qkv, const float* cs, const float* sn, const fl
     long long TT = (long long)T;
     int HH = (int)H, DD = (int)D;
     void* args[12] = {&qkv8, &cs, &sn, &qw, &kw, &eps, &q8, &k8, &v8, &TT, &HH, &DD};
-    const void* fn = dtype == VITATTN_BF16 ? reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true>)
-                                           : reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false>);
+    const bool bf = dtype == VITATTN_BF16;
+    const void* fn =
+        copy_v ? (bf ? reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true, true>)
+                     : reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false, true>))
+               : (bf ? reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true, false>)
+                     : reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false, false>));
     cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(vitattn::kRopeThreads), args, 0, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return VITATTN_OK;
@@ -525,9 +610,10 @@ int checked_run(cudaStream_t stream, Go go) {
 int forward_checked(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
                     int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags,
                     int64_t Hkv = 0, const Ext& ext = Ext()) {
-    int rc = ext.Nk ? check_args_ext(q, k, v, out, ext.lse, B, N, ext.Nk, H, D, scale, dtype)
-             : Hkv  ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
-                    : check_args(q, k, v, out, B, N, H, D, scale, dtype);
+    int rc = ext.ts   ? check_args_strided(q, k, v, out, B, N, H, D, ext.ts, scale, dtype)
+             : ext.Nk ? check_args_ext(q, k, v, out, ext.lse, B, N, ext.Nk, H, D, scale, dtype)
+             : Hkv    ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
+                      : check_args(q, k, v, out, B, N, H, D, scale, dtype);
     if (rc) return rc;
     return checked_run(stream,
                        [&] { return launch(q, k, v, out, B, N, H, D, scale, dtype, stream, flags, Hkv, ext); });
@@ -541,6 +627,97 @@ int forward_varlen_checked(const void* q, const void* k, const void* v, void* ou
     return checked_run(stream, [&] {
         return launch_varlen(q, k, v, out, cu, num_seqs, H, D, scale, dtype, stream, flags);
     });
+}
+
+// ---------------------------------------------------------------- host-buffer entry
+
+// The host-buffer entry splits the batch into up to kHostChunks groups of
+// whole images so that copies and kernels overlap: the inputs of group c+1
+// travel host -> device while the kernel of group c runs and the output of
+// group c-1 travels back.  Two copy streams per (host thread, device) carry
+// the two directions; the kernels run on the caller's stream.
+constexpr int kHostChunks = 8;
+
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr;
+    cudaEvent_t in[kHostChunks] = {}, ran[kHostChunks] = {}, out[kHostChunks] = {};
+};
+thread_local HostPipe t_pipe[kMaxDevices];
+
+int host_pipe(int dev, HostPipe** out) {
+    HostPipe& hp = t_pipe[dev];
+    if (!hp.ready) {
+        cudaError_t e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming);
+        for (int c = 0; c < kHostChunks && e == cudaSuccess; ++c) {
+            e = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.ran[c], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.out[c], cudaEventDisableTiming);
+        }
+        if (e != cudaSuccess) return cuda_fail(e);
+        hp.ready = true;
+    }
+    *out = &hp;
+    return VITATTN_OK;
+}
+
+int forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq, void* dk, void* dv,
+                 void* dout, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int dtype,
+                 cudaStream_t s) {
+    if (!hq || !hk || !hv || !hout) return VITATTN_ERR_NULL;
+    int rc = check_args(dq, dk, dv, dout, B, N, H, D, scale, dtype);
+    if (rc) return rc;
+    int num_sms = 0;
+    rc = device_info(&num_sms);
+    if (rc) return rc;
+    rc = check_device_ptrs({dq, dk, dv, dout});
+    if (rc) return rc;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    HostPipe* hp = nullptr;
+    rc = host_pipe(dev, &hp);
+    if (rc) return rc;
+
+    const int64_t per_chunk = (B + kHostChunks - 1) / kHostChunks;  // images per group
+    const int nchunks = (int)((B + per_chunk - 1) / per_chunk);
+    const size_t image_bytes = (size_t)N * (size_t)H * (size_t)D * 2u;
+    const void* hsrc[3] = {hq, hk, hv};
+    uint8_t* ddst[3] = {static_cast<uint8_t*>(dq), static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv)};
+    // the copies start once the caller's earlier work on `s` is done (it may still read dq..dout)
+    e = cudaEventRecord(hp->start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->h2d, hp->start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->d2h, hp->start, 0);
+    if (e != cudaSuccess) return cuda_fail(e);
+    for (int c = 0; c < nchunks; ++c) {
+        const int64_t b0 = (int64_t)c * per_chunk;
+        const int64_t nb = std::min<int64_t>(per_chunk, B - b0);
+        const size_t off = (size_t)b0 * image_bytes, bytes = (size_t)nb * image_bytes;
+        for (int i = 0; i < 3 && e == cudaSuccess; ++i)
+            e = cudaMemcpyAsync(ddst[i] + off, static_cast<const uint8_t*>(hsrc[i]) + off, bytes,
+                                cudaMemcpyHostToDevice, hp->h2d);
+        if (e == cudaSuccess) e = cudaEventRecord(hp->in[c], hp->h2d);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->in[c], 0);
+        if (e != cudaSuccess) return cuda_fail(e);
+        rc = launch(ddst[0] + off, ddst[1] + off, ddst[2] + off, static_cast<uint8_t*>(dout) + off, nb, N, H, D,
+                    scale, dtype, s, 0);
+        if (rc) return rc;
+        e = cudaEventRecord(hp->ran[c], s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->d2h, hp->ran[c], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(static_cast<uint8_t*>(hout) + off, static_cast<const uint8_t*>(dout) + off, bytes,
+                                cudaMemcpyDeviceToHost, hp->d2h);
+        if (e == cudaSuccess) e = cudaEventRecord(hp->out[c], hp->d2h);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    // work the caller enqueues on `s` afterwards (or a synchronisation of `s`) follows the last
+    // output copy; the copy stream runs in order, so that covers every group
+    e = cudaStreamWaitEvent(s, hp->out[nchunks - 1], 0);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return VITATTN_OK;
 }
 
 }  // namespace
@@ -693,25 +870,62 @@ int vitattn_check_args_qkv_norm_rope(const void* qkv, const float* cos_table, co
     return check_args_norm_rope(qkv, cos_table, sin_table, q_norm_w, k_norm_w, eps, q, k, v, T, H, D, dtype);
 }
 
+int vitattn_forward_strided(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
+                            int64_t H, int64_t D, int64_t q_stride, int64_t k_stride, int64_t v_stride, float scale,
+                            int dtype, vitattn_stream_t stream) {
+    const int64_t ts[3] = {q_stride, k_stride, v_stride};
+    Ext ext;
+    ext.ts = ts;
+    return launch(q, k, v, out, B, N, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), 0, 0, ext);
+}
+
+int vitattn_forward_strided_checked(const void* q, const void* k, const void* v, void* out, int64_t B,
+                                    int64_t N, int64_t H, int64_t D, int64_t q_stride, int64_t k_stride,
+                                    int64_t v_stride, float scale, int dtype, vitattn_stream_t stream) {
+    const int64_t ts[3] = {q_stride, k_stride, v_stride};
+    Ext ext;
+    ext.ts = ts;
+    return forward_checked(q, k, v, out, B, N, H, D, scale, dtype, reinterpret_cast<cudaStream_t>(stream), 0, 0,
+                           ext);
+}
+
+int vitattn_check_args_strided(const void* q, const void* k, const void* v, const void* out, int64_t B, int64_t N,
+                               int64_t H, int64_t D, int64_t q_stride, int64_t k_stride, int64_t v_stride,
+                               float scale, int dtype) {
+    const int64_t ts[3] = {q_stride, k_stride, v_stride};
+    return check_args_strided(q, k, v, out, B, N, H, D, ts, scale, dtype);
+}
+
+int vitattn_qk_rope(const void* qkv, const float* cos_table, const float* sin_table, void* q, void* k, int64_t T,
+                    int64_t H, int64_t D, int dtype, vitattn_stream_t stream) {
+    return launch_rope(qkv, cos_table, sin_table, q, k, nullptr, T, H, D, dtype,
+                       reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+int vitattn_check_args_qk_rope(const void* qkv, const float* cos_table, const float* sin_table, const void* q,
+                               const void* k, int64_t T, int64_t H, int64_t D, int dtype) {
+    return check_args_rope(qkv, cos_table, sin_table, q, k, nullptr, T, H, D, dtype, false);
+}
+
+int vitattn_qk_norm_rope(const void* qkv, const float* cos_table, const float* sin_table, const float* q_norm_w,
+                         const float* k_norm_w, float eps, void* q, void* k, int64_t T, int64_t H, int64_t D,
+                         int dtype, vitattn_stream_t stream) {
+    return launch_norm_rope(qkv, cos_table, sin_table, q_norm_w, k_norm_w, eps, q, k, nullptr, T, H, D, dtype,
+                            reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+int vitattn_check_args_qk_norm_rope(const void* qkv, const float* cos_table, const float* sin_table,
+                                    const float* q_norm_w, const float* k_norm_w, float eps, const void* q,
+                                    const void* k, int64_t T, int64_t H, int64_t D, int dtype) {
+    return check_args_norm_rope(qkv, cos_table, sin_table, q_norm_w, k_norm_w, eps, q, k, nullptr, T, H, D, dtype,
+                                false);
+}
+
 int vitattn_forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq,
                          void* dk, void* dv, void* dout, int64_t B, int64_t N, int64_t H,
                          int64_t D, float scale, int dtype, vitattn_stream_t stream) {
-    if (!hq || !hk || !hv || !hout) return VITATTN_ERR_NULL;
-    int rc = check_args(dq, dk, dv, dout, B, N, H, D, scale, dtype);
-    if (rc) return rc;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const size_t bytes = (size_t)B * (size_t)N * (size_t)H * (size_t)D * 2u;
-    const void* hsrc[3] = {hq, hk, hv};
-    void* ddst[3] = {dq, dk, dv};
-    for (int i = 0; i < 3; ++i) {
-        cudaError_t e = cudaMemcpyAsync(ddst[i], hsrc[i], bytes, cudaMemcpyHostToDevice, s);
-        if (e != cudaSuccess) return cuda_fail(e);
-    }
-    rc = launch(dq, dk, dv, dout, B, N, H, D, scale, dtype, s, 0);
-    if (rc) return rc;
-    cudaError_t e = cudaMemcpyAsync(hout, dout, bytes, cudaMemcpyDeviceToHost, s);
-    if (e != cudaSuccess) return cuda_fail(e);
-    return VITATTN_OK;
+    return forward_host(hq, hk, hv, hout, dq, dk, dv, dout, B, N, H, D, scale, dtype,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 int vitattn_check_args(const void* q, const void* k, const void* v, const void* out, int64_t B,
@@ -731,7 +945,8 @@ const char* vitattn_strerror(int status) {
         case VITATTN_ERR_CUDA: return "CUDA error (see vitattn_last_cuda_error)";
         case VITATTN_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
         case VITATTN_ERR_SCALE: return "scale must be finite (eps: finite and >= 0)";
-        case VITATTN_ERR_DEVICE: return "the current device is not an sm_100 GPU";
+        case VITATTN_ERR_DEVICE:
+            return "the current device is not an sm_100 GPU, or a pointer is not memory its kernels can use";
         case VITATTN_ERR_SEQLENS: return "cu_seqlens must start at 0 and never decrease";
         case VITATTN_ERR_RANGE: return "a bf16 V value has magnitude >= 65536, outside the f16 P.V product's range";
         default: return "unknown status";

@@ -78,6 +78,16 @@ def lib() -> ctypes.CDLL:
         norm_rope = [p, p, p, p, p, f32, p, p, p, i64, i64, i64, i32]
         L.vitattn_qkv_norm_rope.argtypes = norm_rope + [p]
         L.vitattn_check_args_qkv_norm_rope.argtypes = norm_rope
+        strided = [p, p, p, p, i64, i64, i64, i64, i64, i64, i64, f32, i32, p]
+        L.vitattn_forward_strided.argtypes = strided
+        L.vitattn_forward_strided_checked.argtypes = strided
+        L.vitattn_check_args_strided.argtypes = strided[:-1]
+        qk_rope = [p, p, p, p, p, i64, i64, i64, i32]
+        L.vitattn_qk_rope.argtypes = qk_rope + [p]
+        L.vitattn_check_args_qk_rope.argtypes = qk_rope
+        qk_norm_rope = [p, p, p, p, p, f32, p, p, i64, i64, i64, i32]
+        L.vitattn_qk_norm_rope.argtypes = qk_norm_rope + [p]
+        L.vitattn_check_args_qk_norm_rope.argtypes = qk_norm_rope
         L.vitattn_strerror.argtypes = [i32]
         L.vitattn_strerror.restype = ctypes.c_char_p
         for f in (L.vitattn_forward, L.vitattn_forward_checked, L.vitattn_test_forward_flags,
@@ -88,7 +98,9 @@ def lib() -> ctypes.CDLL:
                   L.vitattn_forward_gqa, L.vitattn_forward_gqa_checked, L.vitattn_test_forward_gqa_flags,
                   L.vitattn_check_args_gqa, L.vitattn_forward_ext, L.vitattn_forward_ext_checked,
                   L.vitattn_test_forward_ext_flags, L.vitattn_check_args_ext, L.vitattn_qkv_norm_rope,
-                  L.vitattn_check_args_qkv_norm_rope):
+                  L.vitattn_check_args_qkv_norm_rope, L.vitattn_forward_strided,
+                  L.vitattn_forward_strided_checked, L.vitattn_check_args_strided, L.vitattn_qk_rope,
+                  L.vitattn_check_args_qk_rope, L.vitattn_qk_norm_rope, L.vitattn_check_args_qk_norm_rope):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -128,6 +140,31 @@ def forward_host_ptr(hq, hk, hv, hout, dq, dk, dv, dout, B, N, H, D, scale, dtyp
                                           float(scale), dtype, stream))
 
 
+def _same_device(what: str, *tensors):
+    """Raise ValueError unless every tensor lives on the first one's CUDA device.
+
+    The call runs on that device; a tensor on another GPU would otherwise be
+    read (or written) across devices by the kernel's copies."""
+    dev = tensors[0].device
+    for t in tensors[1:]:
+        if t.device != dev:
+            raise ValueError(f"{what}: every tensor must be on device {dev}, got one on {t.device}")
+
+
+def _stream_handle(stream, device):
+    """The raw cudaStream_t of ``stream`` (None: the device's current stream),
+    refusing a torch stream of another device."""
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, int):
+        return stream
+    if stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
+    return stream.cuda_stream
+
+
 def _dtype_code(t) -> int:
     import torch
 
@@ -164,9 +201,8 @@ def forward(q, k, v, out=None, scale=None, stream=None, checked=False):
         out = torch.empty_like(q)
     elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
         raise ValueError("out must be a contiguous CUDA tensor like q")
-    if stream is None:
-        stream = torch.cuda.current_stream(q.device)
-    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    _same_device("vitattn_forward", q, k, v, out)
+    handle = _stream_handle(stream, q.device)
     with torch.cuda.device(q.device):
         rc = forward_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, D,
                          scale, dtype, handle, checked=checked)
@@ -237,9 +273,8 @@ def forward_varlen(q, k, v, cu_seqlens, out=None, scale=None, stream=None, check
         out = torch.empty_like(q)
     elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
         raise ValueError("out must be a contiguous CUDA tensor like q")
-    if stream is None:
-        stream = torch.cuda.current_stream(q.device)
-    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    _same_device("vitattn_forward_varlen", q, k, v, out)
+    handle = _stream_handle(stream, q.device)
     with torch.cuda.device(q.device):
         rc = forward_varlen_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), cu_seqlens, H, D,
                                 scale, dtype, handle, checked=checked)
@@ -284,10 +319,9 @@ def qkv_rope(qkv, cos, sin, stream=None):
         T *= n
     if tuple(cos.shape) != (T, D) or tuple(sin.shape) != (T, D):
         raise ValueError("cos and sin must be [T, D] with T the token count of qkv")
+    _same_device("vitattn_qkv_rope", qkv, cos, sin)
     q, k, v = (torch.empty(lead + (H, D), dtype=qkv.dtype, device=qkv.device) for _ in range(3))
-    if stream is None:
-        stream = torch.cuda.current_stream(qkv.device)
-    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    handle = _stream_handle(stream, qkv.device)
     with torch.cuda.device(qkv.device):
         rc = qkv_rope_ptr(qkv.data_ptr(), cos.data_ptr(), sin.data_ptr(), q.data_ptr(), k.data_ptr(),
                           v.data_ptr(), T, H, D, dtype, handle)
@@ -334,10 +368,9 @@ def qkv_norm_rope(qkv, cos, sin, q_norm_w, k_norm_w, eps, stream=None):
         raise ValueError("cos and sin must be [T, D] with T the token count of qkv")
     if tuple(q_norm_w.shape) != (D,) or tuple(k_norm_w.shape) != (D,):
         raise ValueError("the norm weights must be [D]")
+    _same_device("vitattn_qkv_norm_rope", *ts)
     q, k, v = (torch.empty(lead + (H, D), dtype=qkv.dtype, device=qkv.device) for _ in range(3))
-    if stream is None:
-        stream = torch.cuda.current_stream(qkv.device)
-    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    handle = _stream_handle(stream, qkv.device)
     with torch.cuda.device(qkv.device):
         rc = qkv_norm_rope_ptr(qkv.data_ptr(), cos.data_ptr(), sin.data_ptr(), q_norm_w.data_ptr(),
                                k_norm_w.data_ptr(), eps, q.data_ptr(), k.data_ptr(), v.data_ptr(), T, H, D,
@@ -387,9 +420,8 @@ def forward_gqa(q, k, v, out=None, scale=None, stream=None, checked=False):
         out = torch.empty_like(q)
     elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
         raise ValueError("out must be a contiguous CUDA tensor like q")
-    if stream is None:
-        stream = torch.cuda.current_stream(q.device)
-    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    _same_device("vitattn_forward_gqa", q, k, v, out)
+    handle = _stream_handle(stream, q.device)
     with torch.cuda.device(q.device):
         rc = forward_gqa_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, Hkv, D, scale,
                              dtype, handle, checked=checked)
@@ -440,10 +472,9 @@ def forward_ext(q, k, v, out=None, scale=None, causal=False, with_lse=False, str
         out = torch.empty_like(q)
     elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
         raise ValueError("out must be a contiguous CUDA tensor like q")
+    _same_device("vitattn_forward_ext", q, k, v, out)
     lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device) if with_lse else None
-    if stream is None:
-        stream = torch.cuda.current_stream(q.device)
-    handle = stream if isinstance(stream, int) else stream.cuda_stream
+    handle = _stream_handle(stream, q.device)
     with torch.cuda.device(q.device):
         rc = forward_ext_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                              lse.data_ptr() if lse is not None else 0, B, Lq, Lk, H, D, scale, causal, dtype,
@@ -451,3 +482,113 @@ def forward_ext(q, k, v, out=None, scale=None, causal=False, with_lse=False, str
     if rc != 0:
         raise VitAttnError(rc, "vitattn_forward_ext")
     return (out, lse) if with_lse else out
+
+
+def check_args_strided(q, k, v, out, B, N, H, D, q_stride, k_stride, v_stride, scale, dtype) -> int:
+    """Status the token-strided argument checks give (pointers as ints); no CUDA call."""
+    return int(lib().vitattn_check_args_strided(q, k, v, out, B, N, H, D, q_stride, k_stride, v_stride,
+                                                float(scale), dtype))
+
+
+def forward_strided_ptr(q, k, v, out, B, N, H, D, q_stride, k_stride, v_stride, scale, dtype, stream=0,
+                        checked=False) -> int:
+    """Raw token-strided call on device pointers (ints); returns the status."""
+    L = lib()
+    args = (q, k, v, out, B, N, H, D, q_stride, k_stride, v_stride, float(scale), dtype, stream)
+    if checked:
+        return int(L.vitattn_forward_strided_checked(*args))
+    return int(L.vitattn_forward_strided(*args))
+
+
+def _token_stride(t, N, H, D, name):
+    """The element stride between tokens of a [B, N, H, D] view whose heads
+    and head dims are dense (e.g. ``qkv[:, :, 0]`` of a [B, N, 3, H, D] tensor)."""
+    st = t.stride()
+    if st[3] != 1 or st[2] != D or st[0] != N * st[1]:
+        raise ValueError(f"{name} must be a [B, N, H, D] view with dense heads and a token stride "
+                         f"(strides {st})")
+    return st[1]
+
+
+def forward_strided(q, k, v, out=None, scale=None, stream=None, checked=False):
+    """Attention on ``[B, N, H, D]`` views whose tokens need not be adjacent:
+    each of q, k, v may be a column range of a packed projection, e.g.
+    ``qkv.unbind(2)`` of a ``[B, N, 3, H, D]`` tensor (token stride 3*H*D),
+    read in place.  ``out`` is a dense ``[B, N, H, D]`` tensor."""
+    import torch
+
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [B, N, H, D] shape")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    dtype = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    B, N, H, D = q.shape
+    ts = [_token_stride(t, N, H, D, n) for t, n in ((q, "q"), (k, "k"), (v, "v"))]
+    if scale is None:
+        scale = 1.0 / float(D) ** 0.5
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    elif out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor of q's shape and dtype")
+    _same_device("vitattn_forward_strided", q, k, v, out)
+    handle = _stream_handle(stream, q.device)
+    with torch.cuda.device(q.device):
+        rc = forward_strided_ptr(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, N, H, D, *ts, scale,
+                                 dtype, handle, checked=checked)
+    if rc != 0:
+        raise VitAttnError(rc, "vitattn_forward_strided")
+    return out
+
+
+def check_args_qk_rope(qkv, cos, sin, q, k, T, H, D, dtype) -> int:
+    """Status the q/k-only prologue's argument checks give (pointers as ints); no CUDA call."""
+    return int(lib().vitattn_check_args_qk_rope(qkv, cos, sin, q, k, T, H, D, dtype))
+
+
+def qk_rope(qkv, cos, sin, q_norm_w=None, k_norm_w=None, eps=None, stream=None):
+    """The prologue without the v copy: rotate q and k of a packed
+    ``[..., 3, H, D]`` projection into new ``[..., H, D]`` tensors (after a
+    per-head RMS norm when ``q_norm_w``, ``k_norm_w`` and ``eps`` are given)
+    and return ``(q, k, v)`` with ``v`` the view ``qkv[..., 2, :, :]`` of the
+    projection itself, ready for :func:`forward_strided`."""
+    import torch
+
+    if qkv.dim() < 4 or qkv.shape[-3] != 3:
+        raise ValueError("qkv must be [..., 3, H, D]")
+    normed = q_norm_w is not None or k_norm_w is not None or eps is not None
+    ts = (qkv, cos, sin) + ((q_norm_w, k_norm_w) if normed else ())
+    if normed and (q_norm_w is None or k_norm_w is None or eps is None):
+        raise ValueError("the normed prologue needs q_norm_w, k_norm_w and eps")
+    if not all(t.is_cuda for t in ts):
+        raise ValueError("qkv, cos, sin (and the norm weights) must be CUDA tensors")
+    if not all(t.is_contiguous() for t in ts):
+        raise ValueError("qkv, cos, sin (and the norm weights) must be contiguous")
+    if any(t.dtype != torch.float32 for t in ts[1:]):
+        raise TypeError("cos, sin and the norm weights must be float32")
+    dtype = _dtype_code(qkv)
+    lead = tuple(qkv.shape[:-3])
+    H, D = qkv.shape[-2], qkv.shape[-1]
+    T = 1
+    for n in lead:
+        T *= n
+    if tuple(cos.shape) != (T, D) or tuple(sin.shape) != (T, D):
+        raise ValueError("cos and sin must be [T, D] with T the token count of qkv")
+    if normed and (tuple(q_norm_w.shape) != (D,) or tuple(k_norm_w.shape) != (D,)):
+        raise ValueError("the norm weights must be [D]")
+    _same_device("vitattn_qk_rope", *ts)
+    q, k = (torch.empty(lead + (H, D), dtype=qkv.dtype, device=qkv.device) for _ in range(2))
+    handle = _stream_handle(stream, qkv.device)
+    L = lib()
+    with torch.cuda.device(qkv.device):
+        if normed:
+            rc = L.vitattn_qk_norm_rope(qkv.data_ptr(), cos.data_ptr(), sin.data_ptr(), q_norm_w.data_ptr(),
+                                        k_norm_w.data_ptr(), float(eps), q.data_ptr(), k.data_ptr(), T, H, D, dtype,
+                                        handle)
+        else:
+            rc = L.vitattn_qk_rope(qkv.data_ptr(), cos.data_ptr(), sin.data_ptr(), q.data_ptr(), k.data_ptr(), T, H,
+                                   D, dtype, handle)
+    if rc != 0:
+        raise VitAttnError(rc, "vitattn_qk_norm_rope" if normed else "vitattn_qk_rope")
+    return q, k, qkv.select(-3, 2)
