@@ -72,7 +72,7 @@ def parse():
                     help="timed steps (default: enough for about 2 s of timed work)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
-                    choices=sorted(synth.WORKLOADS) + sorted(synth.RAGGED) + sorted(synth.PROLOGUE))
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.RAGGED) + sorted(synth.PROLOGUE) + sorted(synth.LAYER))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -565,10 +565,128 @@ def run_prologue(args):
     return 0
 
 
+def run_layer(args):
+    """A ViT layer's attention step from its packed QKV projection: the
+    prologue then the attention, one step each.  ``layer_batched`` copies v
+    through the full prologue; ``layer_packed_batched`` rotates q and k only
+    and lets the attention read v from the projection.  value: attention
+    TFLOP/s over the whole step; the line also gives each kernel's share and
+    the algorithmic bytes moved per step."""
+    w = synth.LAYER[args.workload]
+    if args.impl == "reference":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "layer workloads compare two device paths; the oracle arm runs on the attention workloads"}))
+        return 0
+    import torch
+
+    from vit_bidirectional_attention_b200 import vitattn
+
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    pw = synth.PrologueWorkload(w.name, w.images, w.grid, w.H, w.D, w.dtype, index=w.index)
+    qkv, cs, sn = synth.make_prologue(pw)
+    tdt = torch.bfloat16 if w.dtype == synth.BF16 else torch.float16
+    dqkv = torch.from_numpy(qkv.view(np.int16).copy()).view(tdt).to(dev)
+    dcs, dsn = torch.from_numpy(cs).to(dev), torch.from_numpy(sn).to(dev)
+    q, k, v, out = (torch.empty((w.T, w.H, w.D), dtype=tdt, device=dev) for _ in range(4))
+    stream = torch.cuda.Stream(dev)
+    sh = stream.cuda_stream
+    L = vitattn.lib()
+    hd = w.H * w.D
+    v_src = dqkv.data_ptr() + 2 * hd * 2  # v's columns of the projection
+
+    def prologue():
+        if w.packed:
+            rc = L.vitattn_qk_rope(dqkv.data_ptr(), dcs.data_ptr(), dsn.data_ptr(), q.data_ptr(), k.data_ptr(), w.T,
+                                   w.H, w.D, w.dtype, sh)
+        else:
+            rc = L.vitattn_qkv_rope(dqkv.data_ptr(), dcs.data_ptr(), dsn.data_ptr(), q.data_ptr(), k.data_ptr(),
+                                    v.data_ptr(), w.T, w.H, w.D, w.dtype, sh)
+        if rc:
+            raise vitattn.VitAttnError(rc, "prologue")
+
+    def attention():
+        if w.packed:
+            rc = L.vitattn_forward_strided(q.data_ptr(), k.data_ptr(), v_src, out.data_ptr(), w.images, w.N, w.H, w.D,
+                                           hd, hd, 3 * hd, w.scale, w.dtype, sh)
+        else:
+            rc = L.vitattn_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), w.images, w.N, w.H, w.D,
+                                   w.scale, w.dtype, sh)
+        if rc:
+            raise vitattn.VitAttnError(rc, "attention")
+
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            prologue()
+            attention()
+    stream.synchronize()
+    settle = 0
+    t_w = time.perf_counter()
+    with torch.cuda.stream(stream):
+        while time.perf_counter() - t_w < 1.0:
+            prologue()
+            attention()
+            settle += 1
+            if settle % 16 == 0:
+                stream.synchronize()
+    stream.synchronize()
+    steps = args.steps or 200
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.mark("t_start")
+    with torch.cuda.stream(stream):
+        for e in ev:
+            e[0].record(stream)
+            prologue()
+            e[1].record(stream)
+            attention()
+            e[2].record(stream)
+    stream.synchronize()
+    sampler.mark("t_stop")
+    barrier(world)
+    clocks = sampler.stop()
+    pro_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    att_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    ms_step = max_over_ranks(ev[0][0].elapsed_time(ev[-1][2]), world) / steps
+    peaks, _ = measured_peaks()
+    peak = float(peaks["bf16_tflops"]) if peaks else FALLBACK_PEAK_TFLOPS
+    if rank == 0:
+        per_gpu = w.flops / (ms_step * 1e-3) / 1e12
+        print(json.dumps({
+            "metric": METRIC, "value": w.flops * world / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": synth.DTYPE_NAMES[w.dtype],
+            "data": "synthetic (seeded normals; 2-D rope tables of the patch grid)",
+            "clock_settle_launches": {"launches": 2 * settle, "why": "untimed steps after the warm-up until the "
+                                      "nvidia-smi clock sampler has run for 1 s"},
+            "config": {"workload": w.name, "images": w.images, "grid": list(w.grid), "N": w.N, "H": w.H, "D": w.D,
+                       "packed": w.packed, "global_batch": w.images * world,
+                       "l2": f"{w.io_bytes / 2**20:.0f} MiB moved per step > 126 MiB L2, no flush"},
+            "layer": {"prologue_ms": pro_ms, "attention_ms": att_ms,
+                      "prologue_bytes": w.prologue_bytes, "attention_bytes": w.attention_bytes,
+                      "bytes_per_step": w.io_bytes,
+                      "prologue_gbs": w.prologue_bytes / (pro_ms * 1e-3) / 1e9,
+                      "attention_tflops": w.flops / (att_ms * 1e-3) / 1e12},
+            "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": "TFLOP/s", "frac": per_gpu / peak,
+                         "traffic": None, "kernel": "prologue + vitattn::fwd_kernel_sp",
+                         "note": "whole layer step; the attention kernel alone is layer.attention_tflops"},
+            "gpu_launches": 2 * steps,
+            "clocks": clocks,
+            "cpu_baseline": None,
+        }), flush=True)
+    ranks.finish(world)
+    return 0
+
+
 def main():
     args = parse()
     if args.workload in synth.PROLOGUE:
         return run_prologue(args)
+    if args.workload in synth.LAYER:
+        return run_layer(args)
     if args.impl == "reference":
         return run_reference(args)
     import numpy as np

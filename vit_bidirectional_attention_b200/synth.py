@@ -248,6 +248,69 @@ PROLOGUE = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class LayerWorkload:
+    """The attention step of one ViT layer from its packed QKV projection:
+    the prologue (split + 2-D rope) and the attention, on ``images`` images
+    of ``grid`` patches.  ``packed``: the q/k-only prologue and the attention
+    reading v straight from the projection (token stride 3*H*D); otherwise
+    the full prologue (which copies v) and the dense attention."""
+    name: str
+    images: int
+    grid: tuple
+    H: int
+    D: int
+    dtype: int
+    packed: bool
+    index: int = 0
+
+    @property
+    def seed(self) -> int:
+        return SEED_BASE + self.index
+
+    @property
+    def N(self) -> int:
+        return self.grid[0] * self.grid[1]
+
+    @property
+    def T(self) -> int:
+        return self.images * self.N
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def flops(self) -> float:
+        return 4.0 * self.images * self.H * self.N * self.N * self.D
+
+    @property
+    def prologue_bytes(self) -> int:
+        """The prologue's reads and writes: q and k (and v unless packed) in
+        and out once, plus the two f32 rope tables."""
+        parts = 2 if self.packed else 3
+        return 2 * parts * self.T * self.H * self.D * 2 + 2 * self.T * self.D * 4
+
+    @property
+    def attention_bytes(self) -> int:
+        """q, k, v read once and the output written once."""
+        return 4 * self.T * self.H * self.D * 2
+
+    @property
+    def io_bytes(self) -> int:
+        return self.prologue_bytes + self.attention_bytes
+
+
+LAYER = {
+    w.name: w
+    for w in (
+        # the batched workload's layer (32 images of 32 x 32 patches, 16 heads, D = 64)
+        LayerWorkload("layer_batched", 32, (32, 32), 16, 64, BF16, packed=False, index=6),
+        LayerWorkload("layer_packed_batched", 32, (32, 32), 16, 64, BF16, packed=True, index=6),
+    )
+}
+
+
 def make_prologue(w: PrologueWorkload):
     """(qkv bits [T, 3, H, D], cos [T, D], sin [T, D]) for prologue workload ``w``."""
     qkv = make_qkv_packed(w.T, w.H, w.D, w.dtype, seed=w.seed)
