@@ -150,9 +150,9 @@ VITATTN_API int vitattn_forward_checked(const void* q, const void* k, const void
  *             vitattn_forward); Lq, Lk >= 1.
  *   lse       NULL, or a 16-byte aligned device pointer to [B, H, Lq] float32
  *             receiving log(sum_j exp(scale * q_i . k_j)) over the keys row i
- *             sees (natural log).  The probabilities enter the P.V product
- *             as f16 (see the layout notes above), so lse is that of the
- *             rounded weights: within ~1e-3 of the exact value.
+ *             sees (natural log), from the f32 sum of the probabilities
+ *             (computed with the hardware exp2 approximation): within ~1e-3
+ *             of the exact value.
  *   causal    nonzero: the aligned causal mask above.  A row that sees no key
  *             (only when Lq > Lk) is written as 0 with lse = -inf.
  * Lq = Lk with causal = 0 and lse = NULL is exactly vitattn_forward.

@@ -10,7 +10,9 @@ agents -- the TMA producer, the MMA issuer (tcgen05 operations complete in
 issue order, after arbitrary delays), the softmax warpgroups (a rescale, and
 with it the wait for the previous P.V, happens at random), and the bf16
 V converter -- under random schedules, applying exactly the kernel's parity
-rule, and fails on
+rule.  A softmax warpgroup runs an item's epilogue (wait for O full, release
+O) after handing over the next item's first block, as the kernel does.  It
+fails on
 
 * a wait that passes while its barrier is not exactly one phase past the
   intended one (parity aliasing),
@@ -44,6 +46,7 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
     items, CTAs looping over items or not, bf16 (V converter) or f16.
     Returns the number of scheduling steps."""
     rng = random.Random(seed)
+    kbs = [nkb] * n_my  # key blocks of each item
     ns = NS if T == 2 else min(NS, 2)  # S buffers in use
     track_pv = ns != T                 # the "P.V done" barrier is committed
     VS = KS // 2                       # V slots
@@ -75,18 +78,24 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
                 if loop and k >= NQ:
                     yield ("wait", ("q_empty", qb, t), k // NQ - 1)
                 yield ("tma", ("q_full", qb, t))
-            for _ in range(nkb):
+            for _ in range(kbs[k]):
                 for _kv in range(2):
                     yield ("wait", ("kv_empty", r % KS), r // KS - 1)
                     yield ("tma", ("kv_full", r % KS))
                     r += 1
 
     def mma():
-        total = n_my * T * nkb
+        # units in issue order: (t, j, k, g) for block j of item k, tile t
+        units, g = [], 0
+        for k in range(n_my):
+            for j in range(kbs[k]):
+                for t in range(T):
+                    units.append((t, j, k, g))
+                g += 1
+        total = len(units)
 
         def unit(u):
-            g, t = divmod(u, T)
-            k, j = divmod(g, nkb)
+            t, j, k, g = units[u]
             return t, j, k, g, u % ns
 
         def issue_s(u):
@@ -99,7 +108,7 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
             commits = [("s_full", buf)]
             if t == T - 1:
                 commits.append(("kv_empty", (2 * g) % KS))
-            if loop and j == nkb - 1:
+            if loop and j == kbs[k] - 1:
                 commits.append(("q_empty", qb, t))
             yield ("mma", commits)
 
@@ -118,7 +127,7 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
                 commits.append(("o_ready", t))
             if t == T - 1:
                 commits.append(("kv_empty", (2 * g + 1) % KS))
-            if j == nkb - 1:
+            if j == kbs[k] - 1:
                 commits.append(("o_full", t))
             yield ("mma", commits)
 
@@ -134,20 +143,36 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
 
     def softmax(t):
         g = 0
+        o_phase = 0  # items so far with at least one block
+        pend = None  # (O-full phase, has blocks) of the item whose epilogue is pending
+
+        def finish(pending):
+            phase, has_blocks = pending
+            if has_blocks:
+                yield ("wait", ("o_full", t), phase)
+            if loop:
+                yield ("arrive", ("o_empty", t), 128)
+
         for k in range(n_my):
-            for j in range(nkb):
+            for j in range(kbs[k]):
                 u = T * g + t
                 yield ("wait", ("s_full", u % ns), u // ns)
                 if j > 0 and track_pv and rng.random() < 0.5:  # a row's max grew: rescale O
                     yield ("wait", ("o_ready", t), g - 1)
                 yield ("arrive", ("p_full", t, g & 1), 128)
                 g += 1
-            yield ("wait", ("o_full", t), k)
-            if loop:
-                yield ("arrive", ("o_empty", t), 128)
+                if loop and j == 0 and pend is not None:
+                    yield from finish(pend)
+                    pend = None
+            if loop and pend is not None:  # the item had no blocks
+                yield from finish(pend)
+            pend = (o_phase, kbs[k] > 0)
+            o_phase += kbs[k] > 0
+        if pend is not None:
+            yield from finish(pend)
 
     def converter():
-        for g in range(n_my * nkb):
+        for g in range(sum(kbs)):
             idx = 2 * g + 1
             yield ("wait", ("kv_full", idx % KS), idx // KS)
             yield ("arrive", ("v_ready", g % VS), 64)

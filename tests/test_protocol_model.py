@@ -2,7 +2,8 @@
 schedules (``tests/protocol_model.py``): every configuration the kernel can
 launch -- one or two query tiles, two or three S buffers, one or two Q
 buffers, CTAs looping over items or not, bf16 (with the V converter) or f16 --
-must never let a parity wait pass on the wrong phase and never deadlock."""
+must never let a parity wait pass on the wrong phase and never deadlock.
+Each item's epilogue runs after the next item's first block."""
 import itertools
 
 import pytest
@@ -43,6 +44,30 @@ def test_the_model_catches_a_planted_mistake():
     for seed in range(200):
         try:
             mod.run(2, 3, 1, 8, 1, False, True, seed)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+def test_the_model_catches_an_epilogue_deferred_by_a_whole_item():
+    """Sanity of the checker for the deferred epilogue: running item k's
+    epilogue only after item k + 1 has handed over all its blocks (instead of
+    its first) leaves the next P.V waiting on O-empty while the softmax waits
+    on P.V -- a deadlock the model must report."""
+    import inspect
+    import types
+
+    import protocol_model
+
+    text = inspect.getsource(protocol_model)
+    mutant = text.replace("if loop and j == 0 and pend is not None:", "if False:")
+    assert mutant != text
+    mod = types.ModuleType("protocol_model_mutant2")
+    exec(compile(mutant, "protocol_model_mutant2", "exec"), mod.__dict__)
+    failures = 0
+    for seed in range(50):
+        try:
+            mod.run(1, 2, 1, 4, 3, True, False, seed)
         except AssertionError:
             failures += 1
     assert failures > 0

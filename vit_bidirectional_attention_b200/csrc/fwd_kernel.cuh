@@ -371,17 +371,18 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 // p = 2^(c*s - m) for one block, in f32 (ex2.approx, or the polynomial for
 // some pairs), rounded to f16 and written to TMEM as f16 pairs at tP (64
 // columns), 32 scores at a time.  x <= 8 here (the lazy rescale bound), so
-// p <= 256; f16 keeps p down to 2^-24 (subnormals are kept).  Returns the f32
-// sum of the ROUNDED p: the tensor core multiplies V by exactly these
-// weights, so normalising by their own sum keeps O a true weighted average of
-// V rows (a single dominant key then gives its V row exactly, whatever the
-// rounding of its weight).  Columns at or past `valid` get p = 0.
+// p <= 256; f16 keeps p down to 2^-24 (subnormals are kept).  Returns the sum
+// of the f32 p (before rounding), kept in four f32 partial sums added two at
+// a time (add.f32x2): the rounded weights the tensor core uses differ from
+// these by at most 2^-12 relative each, so O / l is within 2^-12 relative of
+// the weighted average of V rows with the rounded weights.  Summing the
+// rounded halves instead (exact weights, one mixed-precision add each) costs
+// 12-37% of the exponential throughput, measured.  Columns at or past `valid`
+// get p = 0.
 template <bool kPartial>
 __device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], int valid, float c2,
                                                 float neg_m, uint32_t tP) {
-    float acc[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] = 0.f;
+    float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
 #pragma unroll
     for (int q = 0; q < kBlockKeys / 32; ++q) {
         uint32_t pk[16];
@@ -404,11 +405,12 @@ __device__ __forceinline__ float exp_pack_store(const float (&s)[kBlockKeys], in
                 p1 = c + 1 < valid ? p1 : 0.f;
             }
             pk[i] = ptx::pack2<false>(p0, p1);
-            ptx::add_halves<false>(pk[i], acc[2 * (i & 1)], acc[2 * (i & 1) + 1]);
+            if (i & 1) acc1 = ptx::fadd2(acc1, make_float2(p0, p1));
+            else acc0 = ptx::fadd2(acc0, make_float2(p0, p1));
         }
         ptx::tmem_st16(tP + 16 * q, pk);
     }
-    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    return (acc0.x + acc0.y) + (acc1.x + acc1.y);
 }
 
 // One V block (a 128 x DP tile, 16-bit elements, any swizzle: the conversion
@@ -459,41 +461,36 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
     }
 }
 
-// O / l for this thread's row, converted and stored with 16-byte stores.
+// O / l for this thread's row, converted and stored with 16-byte stores.  All
+// DP columns are read out of TMEM first; then, if o_empty is nonzero, that
+// barrier is told that O may be overwritten (the next item's first P.V waits
+// for it) before the conversion and the global stores, which need only
+// registers.
 template <int DP, bool kBF16>
-__device__ __forceinline__ void store_row(uint32_t tO, float inv_l, uint8_t* orow, bool row_ok,
-                                          int D) {
+__device__ __forceinline__ void store_row(uint32_t tO, float inv_l, uint8_t* orow, bool row_ok, int D,
+                                          uint32_t o_empty) {
+    constexpr int NF = DP / 32;
+    constexpr bool kTail = DP % 32 != 0;
+    uint32_t r[NF > 0 ? NF : 1][32];
+    uint32_t rt[16];
 #pragma unroll
-    for (int c = 0; c + 32 <= DP; c += 32) {
-        uint32_t r[32];
-        ptx::tmem_ld32(tO + c, r);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            uint32_t w[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                w[i] = ptx::pack2<kBF16>(__uint_as_float(r[8 * g + 2 * i]) * inv_l,
-                                         __uint_as_float(r[8 * g + 2 * i + 1]) * inv_l);
-            const int col = c + 8 * g;
-            if (row_ok && col + 8 <= D) ptx::st_global_v4(orow + 2 * col, w[0], w[1], w[2], w[3]);
-        }
+    for (int c = 0; c < NF; ++c) ptx::tmem_ld32(tO + 32 * c, r[c]);
+    if (kTail) ptx::tmem_ld16(tO + DP - 16, rt);
+    ptx::tmem_wait_ld();
+    if (o_empty != 0u) {
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(o_empty);
     }
-    if (DP % 32) {
-        constexpr int c = DP - 16;
-        uint32_t r[16];
-        ptx::tmem_ld16(tO + c, r);
-        ptx::tmem_wait_ld();
+    auto col_word = [&](int col) -> float {  // column col of O (compile-time index after unrolling)
+        return __uint_as_float(col < 32 * NF ? r[col >> 5][col & 31] : rt[col - (DP - 16)]);
+    };
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            uint32_t w[4];
+    for (int col = 0; col < DP; col += 8) {
+        uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                w[i] = ptx::pack2<kBF16>(__uint_as_float(r[8 * g + 2 * i]) * inv_l,
-                                         __uint_as_float(r[8 * g + 2 * i + 1]) * inv_l);
-            const int col = c + 8 * g;
-            if (row_ok && col + 8 <= D) ptx::st_global_v4(orow + 2 * col, w[0], w[1], w[2], w[3]);
-        }
+        for (int i = 0; i < 4; ++i)
+            w[i] = ptx::pack2<kBF16>(col_word(col + 2 * i) * inv_l, col_word(col + 2 * i + 1) * inv_l);
+        if (row_ok && col + 8 <= D) ptx::st_global_v4(orow + 2 * col, w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -501,6 +498,221 @@ __device__ __forceinline__ void store_row(uint32_t tO, float inv_l, uint8_t* oro
 __device__ __forceinline__ void store_zero_row(uint8_t* orow, bool row_ok, int D) {
     if (!row_ok) return;
     for (int col = 0; col + 8 <= D; col += 8) ptx::st_global_v4(orow + 2 * col, 0u, 0u, 0u, 0u);
+}
+
+// ---------------------------------------------------------------- work items
+
+// A work item: (b, h, group of query tiles) -- for a ragged batch (segment,
+// h, group).  It attends over the n query rows starting at token tok0 + q0
+// of batch b and the nk keys starting at token tok0.
+struct Item {
+    int b, h, q0, nt, tok0, n, nk;  // n query rows, nk keys (equal except for cross lengths)
+};
+
+// Item i.  Items are numbered so that those of one (b, h) are adjacent and
+// the CTAs running at once share K/V in L2.
+template <bool kVarlen>
+__device__ __forceinline__ Item item_of(const FwdParams& p, const SegTable<kVarlen>& seg, int i) {
+    Item it;
+    int qg;
+    if constexpr (kVarlen) {
+        // the segment whose items contain i: the last s with item0[s] <= i
+        // (an empty segment has no items, so it is never the answer)
+        int lo = 0, hi = seg.n;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (seg.item0[mid] <= i) lo = mid;
+            else hi = mid;
+        }
+        const int local = i - seg.item0[lo];
+        it.h = local / seg.qgroups[lo];
+        qg = local - it.h * seg.qgroups[lo];
+        it.b = 0;
+        it.tok0 = seg.start[lo];
+        it.n = seg.len[lo];
+        it.nk = it.n;
+    } else {
+        qg = i % p.n_qgroups;
+        // with the causal mask a later query group sees more keys: take each
+        // head's longest group first, so the grid's last CTAs are short ones
+        if (p.causal) qg = p.n_qgroups - 1 - qg;
+        const int bh = i / p.n_qgroups;
+        it.h = bh % p.H;
+        it.b = bh / p.H;
+        it.tok0 = 0;
+        it.n = p.N;
+        it.nk = p.Nk;
+    }
+    it.q0 = qg * (p.tiles_per_cta * kTileRows);
+    it.nt = (p.tiles_per_cta == 2 && it.q0 + kTileRows < it.n) ? 2 : 1;
+    return it;
+}
+
+// The CTA's k-th work item: looping CTAs take items blockIdx.x + k * gridDim.x.
+__device__ __forceinline__ int local_item(int k) { return (int)blockIdx.x + k * (int)gridDim.x; }
+
+// Key blocks an item runs over: its keys, and with the causal mask only up to
+// the last key its last query row sees (0 if no row sees any key).
+__device__ __forceinline__ int item_kblocks(const FwdParams& p, const Item& it) {
+    int keys = it.nk;
+    if (p.causal) keys = max(0, min(keys, min(it.q0 + it.nt * kTileRows, it.n) + p.causal_off));
+    return (keys + kBlockKeys - 1) / kBlockKeys;
+}
+
+// ---------------------------------------------------------------- roles
+
+// The TMA producer (one lane): for each of the CTA's items its T Q tiles
+// (Q buffer k % NQ, refilled once the S products of item k - NQ have read
+// it), then K_j and V_j of each key block into ring entries 2g and 2g + 1
+// (slot = entry % kStages, refilled once the MMAs that read the previous
+// occupant have completed).  Before returning it waits (bounded) for every
+// copy it started, so that no copy lands after an abort has ended the CTA.
+// Every item of the CTA has nkb key blocks.
+template <int DP, int NQ, int kStages, bool kLoop, bool kVarlen>
+__device__ __forceinline__ void produce(const FwdParams& p, const SegTable<kVarlen>& seg, uint32_t sQ, uint32_t sKV,
+                                        uint32_t sBar, volatile int* abort_flag, int n_my, int T, int nkb,
+                                        uint64_t tmo) {
+    constexpr int TILE = tile_bytes(DP);
+    constexpr int NCH = chunk_count(DP);
+    auto bar = [&](int i) -> uint32_t { return sBar + 8u * (uint32_t)i; };
+#pragma unroll
+    for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int m = 0; m < 3; ++m) ptx::prefetch_tensormap(&p.maps[m][width_class(chunk_width(DP, c))]);
+    int r = 0;  // K/V ring entries issued so far (K_j, V_j of each item in turn)
+    // last item whose Q tile 0 / tile 1 was issued (two scalars rather than an
+    // array indexed by the tile, which would live in local memory)
+    int q_last0 = -1, q_last1 = -1;
+    bool ok = true;
+    for (int k = 0; k < n_my && ok; ++k) {
+        const Item it = item_of<kVarlen>(p, seg, local_item(k));
+        const int qb = k % NQ;
+        for (int t = 0; t < T && ok; ++t) {
+            // Q buffer qb of tile t was last read by the S products of item k - NQ
+            if (kLoop && k >= NQ &&
+                !wait_one(bar(kBarQEmpty + 2 * qb + t), (uint32_t)((k / NQ) - 1) & 1u, abort_flag, tmo, 12)) {
+                ok = false;
+                break;
+            }
+            ptx::mbar_arrive_expect_tx(bar(kBarQFull + 2 * qb + t), TILE);
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+                ptx::tma_load_4d(sQ + (qb * kTilesPerCta + t) * TILE + 256 * chunk_col(DP, c),
+                                 &p.maps[0][width_class(chunk_width(DP, c))], chunk_col(DP, c), it.h,
+                                 it.tok0 + it.q0 + t * kTileRows, it.b, bar(kBarQFull + 2 * qb + t));
+            if (t == 0) q_last0 = k;
+            else q_last1 = k;
+        }
+
+        for (int j = 0; j < nkb && ok; ++j) {
+            for (int kv = 0; kv < 2; ++kv, ++r) {
+                const int slot = r % kStages;
+                const uint32_t phase = (uint32_t)(r / kStages) & 1u;
+                if (!wait_one(bar(kBarKvEmpty + slot), phase ^ 1u, abort_flag, tmo, 1)) {
+                    ok = false;
+                    break;
+                }
+                if (r == 1 && (p.flags & kFlagSkipFirstVLoad)) continue;  // test-only
+                ptx::mbar_arrive_expect_tx(bar(kBarKvFull + slot), TILE);
+#pragma unroll
+                for (int c = 0; c < NCH; ++c)
+                    ptx::tma_load_4d(sKV + slot * TILE + 256 * chunk_col(DP, c),
+                                     &p.maps[1 + kv][width_class(chunk_width(DP, c))], chunk_col(DP, c),
+                                     it.h / p.kv_group, it.tok0 + j * kBlockKeys, it.b, bar(kBarKvFull + slot));
+            }
+        }
+    }
+    // let every copy this CTA started land before the CTA exits (in a normal
+    // run they all have; after an abort some may not have been waited for).
+    // The last fill of each buffer or slot is its latest phase, so its parity
+    // is unambiguous whether or not it was consumed.
+    const uint64_t drain_ns = 200000000ull;
+    for (int t = 0; t < T; ++t) {
+        const int q_last = t == 0 ? q_last0 : q_last1;
+        for (int k = q_last; k >= 0 && k > q_last - NQ; --k)
+            wait_drain(bar(kBarQFull + 2 * (k % NQ) + t), (uint32_t)(k / NQ) & 1u, drain_ns);
+    }
+    for (int idx = r - 1; idx >= 0 && idx >= r - kStages; --idx) {
+        if ((p.flags & kFlagSkipFirstVLoad) && idx == 1) continue;
+        wait_drain(bar(kBarKvFull + idx % kStages), (uint32_t)(idx / kStages) & 1u, drain_ns);
+    }
+}
+
+// The bf16 V converter (the 64 threads of two warps, ct = 0..63): V_g (ring
+// entry 2g + 1) is converted to f16 in place once it lands, made visible to
+// the tensor core's (async) proxy, and announced on v_ready[g % (kStages/2)]
+// (64 arrivals).  The converter can run at most kStages/2 blocks ahead: V_g's
+// slot is refilled only after the last P.V of the block it held.
+template <int TILE, int kStages>
+__device__ __forceinline__ void convert_v_blocks(uint8_t* kv_tiles, uint32_t sBar, int bar_v_ready,
+                                                 volatile int* abort_flag, int nblocks, uint64_t tmo, int ct) {
+    constexpr int kVSlots = kStages / 2;
+    float vmax = 0.f;
+    for (int g = 0; g < nblocks; ++g) {
+        const int idx = 2 * g + 1;
+        const int slot = idx % kStages;
+        if (!wait_warp(sBar + 8u * (uint32_t)(kBarKvFull + slot), (uint32_t)(idx / kStages) & 1u, abort_flag, tmo, 14))
+            break;
+        vmax = convert_v_tile<TILE>(kv_tiles + slot * TILE, ct, vmax);
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(sBar + 8u * (uint32_t)(bar_v_ready + g % kVSlots));
+    }
+    if (vmax >= 65536.f) atomicOr(&g_vitattn_range, 1u);
+}
+
+// S = Q K^T for one 128 x 128 block (M = 128 query rows, N = 128 keys, K =
+// DP in steps of 16), f32 into TMEM columns [d, d + 128).  Descriptors are
+// built once per column chunk; a K step only adds a constant to the start
+// address field (16-byte units), so the issuing thread spends its time
+// issuing MMAs.
+template <int DP, bool kBF16>
+__device__ __forceinline__ void issue_qk(uint32_t d, uint32_t q_tile, uint32_t k_tile, uint32_t leader) {
+    constexpr int NCH = chunk_count(DP);
+    constexpr uint32_t idS = idesc_f16(kBF16, kBlockKeys, false);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        const int w = chunk_width(DP, c);
+        const uint64_t qd = sdesc(q_tile + 256 * chunk_col(DP, c), 16, 16u * (uint32_t)w, swizzle_code(w));
+        const uint64_t kd = sdesc(k_tile + 256 * chunk_col(DP, c), 16, 16u * (uint32_t)w, swizzle_code(w));
+#pragma unroll
+        for (int kk = 0; kk < w / 16; ++kk)
+            ptx::mma_ss_w(d, qd + 2u * kk, kd + 2u * kk, idS, (c == 0 && kk == 0) ? 0u : 1u, leader);
+    }
+}
+
+// O (+)= P V for one key block (f16 x f16): A = P, 16-bit pairs in TMEM
+// columns [a, a + 64); B = the V tile (MN-major); D = O in TMEM columns
+// [d, d + DP).  The 64-column chunks of V form one MMA with N = 64 * n64 (the
+// second 64-column swizzle atom sits one chunk, 16 KB, further: the leading
+// byte offset); narrower tail chunks get an MMA each.
+template <int DP>
+__device__ __forceinline__ void issue_pv(uint32_t d, uint32_t a, uint32_t v_tile, bool accumulate,
+                                         uint32_t leader) {
+    constexpr int NCH = chunk_count(DP);
+    constexpr int N64 = DP / 64;
+    constexpr int NTAIL = NCH - N64;
+    const uint64_t vd64 = sdesc(v_tile, 128u * 128u, 16u * 64u, swizzle_code(64));
+    uint64_t vdt[NTAIL > 0 ? NTAIL : 1];
+#pragma unroll
+    for (int i = 0; i < NTAIL; ++i) {
+        const int c = N64 + i;
+        const int w = chunk_width(DP, c);
+        vdt[i] = sdesc(v_tile + 256 * chunk_col(DP, c), 256u * (uint32_t)w, 16u * (uint32_t)w, swizzle_code(w));
+    }
+#pragma unroll
+    for (int ks = 0; ks < kBlockKeys / 16; ++ks) {
+        const uint32_t acc = (accumulate || ks > 0) ? 1u : 0u;
+        if (N64 > 0)
+            ptx::mma_ts_w(d, a + (uint32_t)(ks * 8), vd64 + (uint64_t)(2 * 64 * ks), idesc_f16(false, 64 * N64, true),
+                          acc, leader);
+#pragma unroll
+        for (int i = 0; i < NTAIL; ++i) {
+            const int c = N64 + i;
+            const int w = chunk_width(DP, c);
+            ptx::mma_ts_w(d + (uint32_t)chunk_col(DP, c), a + (uint32_t)(ks * 8), vdt[i] + (uint64_t)(2 * w * ks),
+                          idesc_f16(false, w, true), acc, leader);
+        }
+    }
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -536,64 +748,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work items: (b, h, group of query tiles) -- for a ragged batch (segment,
-    // h, group) -- numbered so that the items of one (b, h) are adjacent and
-    // the CTAs running at once share K/V in L2.  An item attends over the n
-    // tokens starting at token tok0 of batch b.  This CTA takes items
-    // blockIdx.x, blockIdx.x + gridDim.x, ...; the host launches fewer CTAs
-    // than items only when every item has the same number of query tiles and
-    // key blocks, so T and nkb below hold for all of this CTA's items.
-    struct Item {
-        int b, h, q0, nt, tok0, n, nk;  // n query rows, nk keys (equal except for cross lengths)
-    };
-    auto item_of = [&](int i) -> Item {
-        Item it;
-        int qg;
-        if constexpr (kVarlen) {
-            // the segment whose items contain i: the last s with item0[s] <= i
-            // (an empty segment has no items, so it is never the answer)
-            int lo = 0, hi = seg.n;
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (seg.item0[mid] <= i) lo = mid;
-                else hi = mid;
-            }
-            const int local = i - seg.item0[lo];
-            it.h = local / seg.qgroups[lo];
-            qg = local - it.h * seg.qgroups[lo];
-            it.b = 0;
-            it.tok0 = seg.start[lo];
-            it.n = seg.len[lo];
-            it.nk = it.n;
-        } else {
-            qg = i % p.n_qgroups;
-            // with the causal mask a later query group sees more keys: take each
-            // head's longest group first, so the grid's last CTAs are short ones
-            if (p.causal) qg = p.n_qgroups - 1 - qg;
-            const int bh = i / p.n_qgroups;
-            it.h = bh % p.H;
-            it.b = bh / p.H;
-            it.tok0 = 0;
-            it.n = p.N;
-            it.nk = p.Nk;
-        }
-        it.q0 = qg * (p.tiles_per_cta * kTileRows);
-        it.nt = (p.tiles_per_cta == 2 && it.q0 + kTileRows < it.n) ? 2 : 1;
-        return it;
-    };
+    // This CTA's k-th item is local_item(k).  The host launches fewer CTAs
+    // than items only when every item has the same number of query tiles (T
+    // below) and of key blocks (nkb: the causal mask runs one CTA per item).
+    auto my_item = [&](int k) -> Item { return item_of<kVarlen>(p, seg, local_item(k)); };
     const int n_my = kLoop ? (p.n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 1;
-    const Item first = item_of(blockIdx.x);
+    const Item first = my_item(0);
     const int T = first.nt;
     // key blocks of this CTA's items; with the causal mask, only up to the last
     // key the item's last query row sees (0 if no row sees any key)
-    int nkb;
-    if (kLoop) {
-        nkb = p.n_kblocks;
-    } else {
-        int keys = first.nk;
-        if (p.causal) keys = max(0, min(keys, min(first.q0 + T * kTileRows, first.n) + p.causal_off));
-        nkb = (keys + kBlockKeys - 1) / kBlockKeys;
-    }
+    const int nkb = kLoop ? p.n_kblocks : item_kblocks(p, first);
     const uint64_t tmo = p.timeout_ns;
 
     if (threadIdx.x == 0) {
@@ -633,76 +797,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     ptx::setmaxnreg_dec<kSideRegs>();
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-#pragma unroll
-            for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                for (int m = 0; m < 3; ++m)
-                    ptx::prefetch_tensormap(&p.maps[m][width_class(chunk_width(DP, c))]);
-            int r = 0;         // K/V ring entries issued so far (K_j, V_j of each item in turn)
-            // last item whose Q tile 0 / tile 1 was issued (two scalars rather than an
-            // array indexed by the tile, which would live in local memory)
-            int q_last0 = -1, q_last1 = -1;
-            bool ok = true;
-            for (int k = 0; k < n_my && ok; ++k) {
-                const Item it = item_of((int)blockIdx.x + k * (int)gridDim.x);
-                const int qb = k % NQ;
-                for (int t = 0; t < T && ok; ++t) {
-                    // Q buffer qb of tile t was last read by the S products of item k - NQ
-                    if (kLoop && k >= NQ &&
-                        !wait_one(bar(kBarQEmpty + 2 * qb + t), (uint32_t)((k / NQ) - 1) & 1u, abort_flag,
-                                  tmo, 12)) {
-                        ok = false;
-                        break;
-                    }
-                    ptx::mbar_arrive_expect_tx(bar(kBarQFull + 2 * qb + t), TILE);
-#pragma unroll
-                    for (int c = 0; c < NCH; ++c)
-                        ptx::tma_load_4d(sQ + (qb * kTilesPerCta + t) * TILE + 256 * chunk_col(DP, c),
-                                         &p.maps[0][width_class(chunk_width(DP, c))], chunk_col(DP, c),
-                                         it.h, it.tok0 + it.q0 + t * kTileRows, it.b,
-                                         bar(kBarQFull + 2 * qb + t));
-                    if (t == 0) q_last0 = k;
-                    else q_last1 = k;
-                }
-
-                for (int j = 0; j < nkb && ok; ++j) {
-                    for (int kv = 0; kv < 2; ++kv, ++r) {
-                        const int slot = r % kStages;
-                        const uint32_t phase = (uint32_t)(r / kStages) & 1u;
-                        if (!wait_one(bar(kBarKvEmpty + slot), phase ^ 1u, abort_flag, tmo, 1)) {
-                            ok = false;
-                            break;
-                        }
-                        if (r == 1 && (p.flags & kFlagSkipFirstVLoad)) continue;  // test-only
-                        ptx::mbar_arrive_expect_tx(bar(kBarKvFull + slot), TILE);
-#pragma unroll
-                        for (int c = 0; c < NCH; ++c)
-                            ptx::tma_load_4d(sKV + slot * TILE + 256 * chunk_col(DP, c),
-                                             &p.maps[1 + kv][width_class(chunk_width(DP, c))],
-                                             chunk_col(DP, c), it.h / p.kv_group, it.tok0 + j * kBlockKeys,
-                                             it.b, bar(kBarKvFull + slot));
-                    }
-                }
-            }
-            {
-                // let every copy this CTA started land before the CTA exits (in a
-                // normal run they all have; after an abort some may not have been
-                // waited for).  The last fill of each buffer or slot is its latest
-                // phase, so its parity is unambiguous whether or not it was consumed.
-                const uint64_t drain_ns = 200000000ull;
-                for (int t = 0; t < T; ++t) {
-                    const int q_last = t == 0 ? q_last0 : q_last1;
-                    for (int k = q_last; k >= 0 && k > q_last - NQ; --k)
-                        wait_drain(bar(kBarQFull + 2 * (k % NQ) + t), (uint32_t)(k / NQ) & 1u, drain_ns);
-                }
-                for (int idx = r - 1; idx >= 0 && idx >= r - kStages; --idx) {
-                    if ((p.flags & kFlagSkipFirstVLoad) && idx == 1) continue;
-                    wait_drain(bar(kBarKvFull + idx % kStages), (uint32_t)(idx / kStages) & 1u,
-                               drain_ns);
-                }
-            }
-        }
+        if (lane == 0)
+            produce<DP, NQ, kStages, kLoop, kVarlen>(p, seg, sQ, sKV, sBar, abort_flag, n_my, T, nkb, tmo);
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -710,59 +806,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         // stay warp-uniform); one elected lane issues each MMA and commit.
         {
             const uint32_t leader = ptx::elect_one();
-            // Descriptors are built once per chunk and phase; a K step then
-            // only adds a constant to the start-address field (16-byte units),
-            // so the single issuing thread spends its time issuing MMAs.
-            constexpr uint32_t idS = idesc_f16(kBF16, kBlockKeys, false);
             constexpr int NS = s_buffers(DP);
             constexpr int OC = o_cols(DP);
             auto mma_s = [&](int qtile, int slot, int buf) {
-                const uint32_t d = tmem + (uint32_t)(buf * kBlockKeys);
-#pragma unroll
-                for (int c = 0; c < NCH; ++c) {
-                    const int w = chunk_width(DP, c);
-                    const uint64_t qd = sdesc(sQ + qtile * TILE + 256 * chunk_col(DP, c), 16,
-                                              16u * (uint32_t)w, swizzle_code(w));
-                    const uint64_t kd = sdesc(sKV + slot * TILE + 256 * chunk_col(DP, c), 16,
-                                              16u * (uint32_t)w, swizzle_code(w));
-#pragma unroll
-                    for (int kk = 0; kk < w / 16; ++kk)
-                        ptx::mma_ss_w(d, qd + 2u * kk, kd + 2u * kk, idS,
-                                      (c == 0 && kk == 0) ? 0u : 1u, leader);
-                }
+                issue_qk<DP, kBF16>(tmem + (uint32_t)(buf * kBlockKeys), sQ + qtile * TILE, sKV + slot * TILE, leader);
             };
-            // P.V (f16 x f16): the 64-column chunks of V form one MMA with N = 64 * n64 (the
-            // second 64-column swizzle atom sits one chunk, 16 KB, further: the
-            // leading byte offset); narrower tail chunks get an MMA each.
-            constexpr int N64 = DP / 64;
-            constexpr int NTAIL = NCH - N64;
             auto mma_pv = [&](int t, int slot, int buf, bool accumulate) {
-                const uint32_t d = tmem + (uint32_t)(NS * kBlockKeys + t * OC);
-                const uint32_t a = tmem + (uint32_t)(buf * kBlockKeys);
-                const uint32_t vbase = sKV + slot * TILE;
-                const uint64_t vd64 = sdesc(vbase, 128u * 128u, 16u * 64u, swizzle_code(64));
-                uint64_t vdt[NTAIL > 0 ? NTAIL : 1];
-#pragma unroll
-                for (int i = 0; i < NTAIL; ++i) {
-                    const int c = N64 + i;
-                    const int w = chunk_width(DP, c);
-                    vdt[i] = sdesc(vbase + 256 * chunk_col(DP, c), 256u * (uint32_t)w,
-                                   16u * (uint32_t)w, swizzle_code(w));
-                }
-#pragma unroll
-                for (int ks = 0; ks < kBlockKeys / 16; ++ks) {
-                    const uint32_t acc = (accumulate || ks > 0) ? 1u : 0u;
-                    if (N64 > 0)
-                        ptx::mma_ts_w(d, a + (uint32_t)(ks * 8), vd64 + (uint64_t)(2 * 64 * ks),
-                                      idesc_f16(false, 64 * N64, true), acc, leader);
-#pragma unroll
-                    for (int i = 0; i < NTAIL; ++i) {
-                        const int c = N64 + i;
-                        const int w = chunk_width(DP, c);
-                        ptx::mma_ts_w(d + (uint32_t)chunk_col(DP, c), a + (uint32_t)(ks * 8),
-                                      vdt[i] + (uint64_t)(2 * w * ks), idesc_f16(false, w, true), acc, leader);
-                    }
-                }
+                issue_pv<DP>(tmem + (uint32_t)(NS * kBlockKeys + t * OC), tmem + (uint32_t)(buf * kBlockKeys),
+                             sKV + slot * TILE, accumulate, leader);
             };
             // K_j and V_j occupy ring entries 2j and 2j+1 (the producer's order).
             auto kv_slot = [](int idx) { return idx % kStages; };
@@ -773,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             // A cursor walks the units s = T*j + t in order, keeping (t, j) and the
             // S buffer s mod ns without divisions (this thread is on the critical path).
             struct Cursor {
-                int t, j, k, g, buf;  // tile, block, item (local index), block count g = k*nkb + j
+                int t, j, k, g, buf;  // tile, block, item (local index), block count g = k*nkb + j, S buffer
             };
             auto advance = [&](Cursor& c) {
                 if (++c.t == T) {
@@ -860,21 +911,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         __syncwarp();
     } else if (kBF16) {
         // ------------------------------------------------------------ V converter (bf16)
-        // V_g (ring entry 2g+1) is converted in place once it lands; both
-        // warps then signal V-ready for it (64 arrivals).
-        const int ct = threadIdx.x - kConvWarp * 32;
-        const int nblocks = n_my * nkb;
-        float vmax = 0.f;
-        for (int g = 0; g < nblocks; ++g) {
-            const int idx = 2 * g + 1;
-            const int slot = idx % kStages;
-            if (!wait_warp(bar(kBarKvFull + slot), (uint32_t)(idx / kStages) & 1u, abort_flag, tmo, 14))
-                break;
-            vmax = convert_v_tile<TILE>(base_ptr + (sKV - base) + slot * TILE, ct, vmax);
-            ptx::fence_proxy_async_smem();
-            ptx::mbar_arrive(bar(kBarVReady + g % kVSlots));
-        }
-        if (vmax >= 65536.f) atomicOr(&g_vitattn_range, 1u);
+        convert_v_blocks<TILE, kStages>(base_ptr + (sKV - base), sBar, kBarVReady, abort_flag, n_my * nkb, tmo,
+                                        (int)threadIdx.x - kConvWarp * 32);
     }
     } else {
         ptx::setmaxnreg_inc<kSoftmaxRegs>();
@@ -894,12 +932,42 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             // both advance by T units per block.
             int sbuf = t % ns, sphase = t / ns;
             int g = 0;
+            int o_phase = 0;  // items so far whose O_t has been (or is being) accumulated
+            // The epilogue of item k (wait for its last P.V, read O_t out, store
+            // O / l) runs after the first block of item k + 1 has been handed to
+            // the MMA warp, so that the last P.V's latency is hidden behind that
+            // block's softmax; O_t is released before the global stores.
+            auto finish = [&](int k, float m_used, float l, int kb, int phase) -> bool {
+                if (kb > 0 && !wait_warp(bar(kBarOFull + t), (uint32_t)phase & 1u, abort_flag, tmo, 8)) return false;
+                ptx::tc_fence_after();
+                const Item it = my_item(k);
+                const int row = it.q0 + t * kTileRows + wq * 32 + lane;
+                uint8_t* orow =
+                    reinterpret_cast<uint8_t*>(p.out) +
+                    ((((size_t)it.b * p.N + (size_t)it.tok0 + (size_t)min(row, it.n - 1)) * p.H + it.h) * p.D) * 2;
+                const uint32_t o_empty = kLoop ? bar(kBarOEmpty + t) : 0u;
+                // a row that saw no key (causal, more queries than keys) is 0
+                if (kb > 0) {
+                    store_row<DP, kBF16>(tO, l > 0.f ? 1.f / l : 0.f, orow, row < it.n, p.D, o_empty);
+                } else {
+                    store_zero_row(orow, row < it.n, p.D);
+                    if (kLoop) ptx::mbar_arrive(o_empty);
+                }
+                if (p.lse != nullptr && row < it.n)
+                    p.lse[((size_t)it.b * p.H + it.h) * p.N + it.tok0 + row] =
+                        l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                return true;
+            };
+            // the item whose epilogue is pending (-1: none) and its row state
+            int pend = -1, pend_kb = 0, pend_phase = 0;
+            float pend_m = 0.f, pend_l = 0.f;
             for (int k = 0; k < n_my && ok; ++k) {
-            const Item it = item_of((int)blockIdx.x + k * (int)gridDim.x);
+            const Item it = my_item(k);
+            const int kb = nkb;
             const int row = it.q0 + t * kTileRows + wq * 32 + lane;
             float m_used = -INFINITY;
             float l = 0.f;
-            for (int j = 0; j < nkb; ++j, ++g) {
+            for (int j = 0; j < kb; ++j, ++g) {
                 const uint32_t tS = tmem + lane_base + (uint32_t)(sbuf * kBlockKeys);
                 const uint32_t s_bar = bar(kBarSFull + sbuf);
                 const uint32_t s_par = (uint32_t)sphase & 1u;
@@ -961,27 +1029,29 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(bar(kBarPFull + 2 * t + (g & 1)));
-            }
-            if (ok && nkb > 0) ok = wait_warp(bar(kBarOFull + t), (uint32_t)k & 1u, abort_flag, tmo, 8);
-            if (ok) {
-                ptx::tc_fence_after();
-                uint8_t* orow =
-                    reinterpret_cast<uint8_t*>(p.out) +
-                    ((((size_t)it.b * p.N + (size_t)it.tok0 + (size_t)min(row, it.n - 1)) * p.H + it.h) * p.D) * 2;
-                // a row that saw no key (causal, more queries than keys) is 0
-                if (nkb > 0) store_row<DP, kBF16>(tO, l > 0.f ? 1.f / l : 0.f, orow, row < it.n, p.D);
-                else store_zero_row(orow, row < it.n, p.D);
-                if (p.lse != nullptr && row < it.n)
-                    p.lse[((size_t)it.b * p.H + it.h) * p.N + it.tok0 + row] =
-                        l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
-                // O_t has been read (store_row waits for each load): the next
-                // item's first P.V may overwrite it
-                if (kLoop) {
-                    ptx::tc_fence_before();
-                    ptx::mbar_arrive(bar(kBarOEmpty + t));
+                // the previous item's epilogue (its O_t is released before this
+                // item's first P.V can start)
+                if (kLoop && j == 0 && pend >= 0) {
+                    ok = finish(pend, pend_m, pend_l, pend_kb, pend_phase);
+                    pend = -1;
+                    if (!ok) break;
                 }
             }
+            if (!ok) break;
+            // an item without key blocks has nothing for its epilogue to wait for
+            if (kLoop && pend >= 0) {
+                ok = finish(pend, pend_m, pend_l, pend_kb, pend_phase);
+                pend = -1;
+                if (!ok) break;
             }
+            pend = k;
+            pend_m = m_used;
+            pend_l = l;
+            pend_kb = kb;
+            pend_phase = o_phase;
+            if (kb > 0) ++o_phase;
+            }
+            if (ok && pend >= 0) ok = finish(pend, pend_m, pend_l, pend_kb, pend_phase);
         }
     }
 
@@ -992,5 +1062,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
 }
+
 
 }  // namespace vitattn

@@ -469,7 +469,9 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     // blocks) for the per-CTA start-up and epilogue to matter, and every item
     // has the same number of query tiles (all have two unless the last group
     // of a head is a single tile); otherwise one CTA per item.
-    // (the causal mask gives items different key-block counts: one CTA per item)
+    // The causal mask gives items different key-block counts, so it runs one
+    // CTA per item, each (b, h)'s longest item first: the hardware's block
+    // scheduler then hands the short items to whichever SM frees up first.
     const bool uniform = !prm.causal && (prm.tiles_per_cta == 1 || (N % 256 == 0 || N % 256 > 128));
     unsigned grid = (unsigned)prm.n_items;
     if (uniform && prm.n_items > num_sms && prm.n_kblocks <= 32) grid = (unsigned)num_sms;
