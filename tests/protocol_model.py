@@ -40,11 +40,15 @@ class Barrier:
             self.ph += 1
 
 
-def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
+def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4, split=False):
     """One random schedule of one CTA: T query tiles (1 or 2), NS S buffers
     (2 or 3, as TMEM allows), NQ Q buffers, nkb key blocks per item, n_my
     items, CTAs looping over items or not, bf16 (V converter) or f16.
-    Returns the number of scheduling steps."""
+    split: one item whose two "tiles" are the two halves of one query tile's
+    key blocks (T = 2, no loop): every unit has its own K/V pair, and the
+    lower half merges the upper half's result at the end.  Returns the
+    number of scheduling steps."""
+    assert not split or (T == 2 and not loop and n_my == 1)
     rng = random.Random(seed)
     kbs = [nkb] * n_my  # key blocks of each item
     ns = NS if T == 2 else min(NS, 2)  # S buffers in use
@@ -69,6 +73,7 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
     for t in range(2):
         B(("p_full", t, 0), 128), B(("p_full", t, 1), 128)
         B(("o_ready", t)), B(("o_full", t)), B(("o_empty", t), 128)
+    B(("merge",), 128)
 
     def loader():
         r = 0
@@ -78,7 +83,7 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
                 if loop and k >= NQ:
                     yield ("wait", ("q_empty", qb, t), k // NQ - 1)
                 yield ("tma", ("q_full", qb, t))
-            for _ in range(kbs[k]):
+            for _ in range(kbs[k] * (T if split else 1)):
                 for _kv in range(2):
                     yield ("wait", ("kv_empty", r % KS), r // KS - 1)
                     yield ("tma", ("kv_full", r % KS))
@@ -98,35 +103,40 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
             t, j, k, g = units[u]
             return t, j, k, g, u % ns
 
+        def pair(t, g):  # the K/V pair a unit reads: its block's, or its own (split)
+            return T * g + t if split else g
+
         def issue_s(u):
             t, j, k, g, buf = unit(u)
             qb = k % NQ
             if j == 0:
                 yield ("wait", ("q_full", qb, t), k // NQ)
-            if t == 0:
-                yield ("wait", ("kv_full", (2 * g) % KS), (2 * g) // KS)
+            e = pair(t, g)
+            if split or t == 0:
+                yield ("wait", ("kv_full", (2 * e) % KS), (2 * e) // KS)
             commits = [("s_full", buf)]
-            if t == T - 1:
-                commits.append(("kv_empty", (2 * g) % KS))
+            if split or t == T - 1:
+                commits.append(("kv_empty", (2 * e) % KS))
             if loop and j == kbs[k] - 1:
                 commits.append(("q_empty", qb, t))
             yield ("mma", commits)
 
         def issue_pv(u):
             t, j, k, g, _ = unit(u)
-            if t == 0:
+            e = pair(t, g)
+            if split or t == 0:
                 if bf16:
-                    yield ("wait", ("v_ready", g % VS), g // VS)
+                    yield ("wait", ("v_ready", e % VS), e // VS)
                 else:
-                    yield ("wait", ("kv_full", (2 * g + 1) % KS), (2 * g + 1) // KS)
+                    yield ("wait", ("kv_full", (2 * e + 1) % KS), (2 * e + 1) // KS)
             if loop and j == 0 and k > 0:
                 yield ("wait", ("o_empty", t), k - 1)
             yield ("wait", ("p_full", t, g & 1), g >> 1)
             commits = []
             if track_pv:
                 commits.append(("o_ready", t))
-            if t == T - 1:
-                commits.append(("kv_empty", (2 * g + 1) % KS))
+            if split or t == T - 1:
+                commits.append(("kv_empty", (2 * e + 1) % KS))
             if j == kbs[k] - 1:
                 commits.append(("o_full", t))
             yield ("mma", commits)
@@ -150,6 +160,12 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
             phase, has_blocks = pending
             if has_blocks:
                 yield ("wait", ("o_full", t), phase)
+            if split:
+                if t == 1:
+                    yield ("arrive", ("merge",), 128)
+                else:
+                    yield ("wait", ("o_full", 1), 0)
+                    yield ("wait", ("merge",), 0)
             if loop:
                 yield ("arrive", ("o_empty", t), 128)
 
@@ -172,7 +188,7 @@ def run(T, NS, NQ, nkb, n_my, loop, bf16, seed, KS=4):
             yield from finish(pend)
 
     def converter():
-        for g in range(sum(kbs)):
+        for g in range(sum(kbs) * (T if split else 1)):
             idx = 2 * g + 1
             yield ("wait", ("kv_full", idx % KS), idx // KS)
             yield ("arrive", ("v_ready", g % VS), 64)

@@ -25,6 +25,17 @@ def test_protocol_has_no_aliasing_or_deadlock(T, NS, NQ, loop, bf16):
                 run(T, NS, NQ, nkb, n_my, loop, bf16, seed)
 
 
+@pytest.mark.parametrize("KS", [4, 6, 8])
+@pytest.mark.parametrize("NS,bf16", [(2, False), (2, True), (3, False), (3, True)])
+def test_split_items_have_no_aliasing_or_deadlock(NS, bf16, KS):
+    """A split item: both softmax warpgroups on one query tile, each over its
+    half of the key blocks with its own K/V pair per unit, merged at the
+    end; with the 4-, 6- and 8-slot rings split items use."""
+    for nkb in (1, 2, 3, 4, 7):
+        for seed in range(16):
+            run(2, NS, 1, nkb, 1, False, bf16, seed, KS=KS, split=True)
+
+
 def test_the_model_catches_a_planted_mistake():
     """Sanity of the checker itself: with a single "P written" barrier per
     tile instead of one per block parity, some schedule lets a softmax run two
@@ -68,6 +79,32 @@ def test_the_model_catches_an_epilogue_deferred_by_a_whole_item():
     for seed in range(50):
         try:
             mod.run(1, 2, 1, 4, 3, True, False, seed)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
+
+
+def test_the_model_catches_a_split_item_sharing_k_blocks():
+    """Sanity of the split model: releasing a split unit's K only after the
+    upper half's S (as for shared blocks) while both halves wait for their
+    own K leaves the producer short of free slots -- or lets a release land
+    on the wrong entry -- and the model must report it."""
+    import inspect
+    import types
+
+    import protocol_model
+
+    text = inspect.getsource(protocol_model)
+    mutant = text.replace("""            if split or t == T - 1:
+                commits.append(("kv_empty", (2 * e) % KS))""", """            if t == T - 1:
+                commits.append(("kv_empty", (2 * e) % KS))""")
+    assert mutant != text
+    mod = types.ModuleType("protocol_model_mutant3")
+    exec(compile(mutant, "protocol_model_mutant3", "exec"), mod.__dict__)
+    failures = 0
+    for seed in range(50):
+        try:
+            mod.run(2, 2, 1, 4, 1, False, False, seed, split=True)
         except AssertionError:
             failures += 1
     assert failures > 0

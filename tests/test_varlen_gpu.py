@@ -20,6 +20,7 @@ MAX_ABS = 1e-2
 REL_FROB = 4e-3
 FORCE_TWO_TILES = 2
 FORCE_ONE_TILE = 4
+NO_SPLIT = 16  # ragged batches never split a tile's key blocks; keep the dense call alike
 
 
 def to_dev(bits, dtype):
@@ -92,7 +93,8 @@ def test_many_short_segments(cuda_device):
 @pytest.mark.parametrize("tiles", [FORCE_TWO_TILES, FORCE_ONE_TILE])
 def test_equal_segments_match_the_dense_entry_bitwise(cuda_device, tiles):
     """B images of N tokens each, packed, give exactly what the dense [B, N, H, D]
-    call gives: keys past an image are masked to probability 0 in both."""
+    call gives: keys past an image are masked to probability 0 in both (the
+    dense call with its key blocks unsplit, as ragged batches run)."""
     import torch
 
     B, N, H, D = 3, 300, 2, 64
@@ -100,7 +102,7 @@ def test_equal_segments_match_the_dense_entry_bitwise(cuda_device, tiles):
     tq, tk, tv = (to_dev(x, synth.BF16) for x in (q, k, v))
     dense = torch.empty_like(tq)
     rc = vitattn.forward_ptr(tq.data_ptr(), tk.data_ptr(), tv.data_ptr(), dense.data_ptr(), B, N, H, D, 0.125,
-                             synth.BF16, torch.cuda.current_stream().cuda_stream, flags=tiles)
+                             synth.BF16, torch.cuda.current_stream().cuda_stream, flags=tiles | NO_SPLIT)
     assert rc == 0
     packed = run_varlen(q.reshape(B * N, H, D), k.reshape(B * N, H, D), v.reshape(B * N, H, D),
                         [0, N, 2 * N, 3 * N], 0.125, synth.BF16, flags=tiles)

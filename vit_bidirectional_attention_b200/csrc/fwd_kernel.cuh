@@ -82,7 +82,7 @@ namespace vitattn {
 constexpr int kTileRows = 128;    // query rows per tile = TMEM lanes
 constexpr int kBlockKeys = 128;   // keys per K/V block
 constexpr int kTilesPerCta = 2;
-constexpr int kMaxStages = 4;     // K/V ring slots (K_j, V_j, K_j+1, V_j+1)
+constexpr int kMaxStages = 8;     // K/V ring slots at most (K in even slots, V in odd ones)
 constexpr int kThreads = 384;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
@@ -116,7 +116,8 @@ constexpr int kBarOFull = kBarOReady + 2;            // [2] per tile: the item's
 constexpr int kBarOEmpty = kBarOFull + 2;            // [2] per tile: the epilogue has read O
 constexpr int kBarVReady = kBarOEmpty + 2;           // [kMaxStages / 2] bf16: the V slot's block is f16
 constexpr int kBarDrain = kBarVReady + kMaxStages / 2;  // [1]
-constexpr int kNumBars = kBarDrain + 1;
+constexpr int kBarMerge = kBarDrain + 1;             // [1] split items: the upper key half's (m, l) are written
+constexpr int kNumBars = kBarMerge + 1;
 
 // Status codes written to g_vitattn_status (0 = fine).
 constexpr unsigned kStatusTimeoutBase = 0x100;  // + site id
@@ -129,6 +130,12 @@ constexpr int kFlagSkipFirstVLoad = 1;
 constexpr int kFlagForceTwoTiles = 2;
 constexpr int kFlagForceOneTile = 4;
 constexpr int kFlagTinyGrid = 8;
+// Test-only host flags: never split a query tile's key blocks over the two
+// softmax warpgroups (see FwdParams::split), or split them from two key
+// blocks on (by default from four: with fewer the merge costs what the
+// shorter chain saves, measured on the 196-token block).
+constexpr int kFlagNoSplit = 16;
+constexpr int kFlagSplitFromTwo = 32;
 
 // ---------------------------------------------------------------- column chunks
 
@@ -171,12 +178,32 @@ __host__ __device__ constexpr bool pv_done_needed(int ns, int ntiles) { return n
 // one runs) when a CTA loops over items and that fits in shared memory, i.e.
 // up to DP = 112.
 __host__ __device__ constexpr int q_buffers(int dp, bool loop) { return (loop && dp <= 112) ? 2 : 1; }
-// K/V ring slots for a padded head dim (even: K in even slots, V in odd ones).
-__host__ __device__ constexpr int kv_stages(int dp) { return kMaxStages; }
-static_assert(kMaxStages % 2 == 0, "K and V alternate in the ring");
-__host__ __device__ constexpr int smem_bytes(int dp, bool loop) {
-    return (q_buffers(dp, loop) * kTilesPerCta + kv_stages(dp)) * tile_bytes(dp) + kNumBars * 8 + 16 + 1024;
+// K/V ring slots (even: K in even slots, V in odd ones).  Four hold two key
+// blocks, each shared by the item's two tiles.  A split item's tiles read
+// different blocks, so a step of both tiles fills four slots by itself: its
+// ring is as deep as shared memory allows (eight slots up to DP = 80, six up
+// to 112), so that the next step's blocks load during this one.
+__host__ __device__ constexpr int kv_stages(int dp, bool split = false) {
+    return split ? (dp <= 80 ? 8 : dp <= 112 ? 6 : 4) : 4;
 }
+static_assert(kMaxStages % 2 == 0, "K and V alternate in the ring");
+static_assert(kv_stages(16, true) <= kMaxStages && kv_stages(128) <= kMaxStages, "ring barriers");
+// Split items exchange one (m, l) pair per query row through shared memory.
+constexpr int kMergeBytes = kTileRows * 2 * 4;
+__host__ __device__ constexpr int smem_bytes(int dp, bool loop, bool split = false) {
+    return (q_buffers(dp, loop) * kTilesPerCta + kv_stages(dp, split)) * tile_bytes(dp) + kNumBars * 8 + 16 +
+           (split ? kMergeBytes : 0) + 1024;
+}
+// Every launchable configuration fits the 227 KB of dynamic shared memory a
+// block may opt into.
+__host__ __device__ constexpr bool smem_fits() {
+    for (int dp = 16; dp <= 128; dp += 16)
+        if (smem_bytes(dp, false) > 227 * 1024 || smem_bytes(dp, true) > 227 * 1024 ||
+            smem_bytes(dp, false, true) > 227 * 1024)
+            return false;
+    return true;
+}
+static_assert(smem_fits(), "shared memory of every configuration");
 
 // Ragged batches (several images' tokens packed along one axis, start
 // offsets cu_seqlens): segment s is tokens start[s] .. start[s] + len[s] - 1,
@@ -210,6 +237,8 @@ struct alignas(64) FwdParams {
     int causal;         // nonzero: query i sees keys j <= i + causal_off only (aligned causal mask)
     int causal_off;     // Nk - N
     float* lse;         // optional [B, H, N] f32: log sum_j exp(scale * q_i . k_j); nullptr: not written
+    int split;          // nonzero: a work item is ONE query tile whose key blocks are split in two halves,
+                        // one per softmax warpgroup, merged at the end (grids too small to fill the SMs)
     float scale_log2;
     int flags;
     unsigned long long timeout_ns;
@@ -494,6 +523,44 @@ __device__ __forceinline__ void store_row(uint32_t tO, float inv_l, uint8_t* oro
     }
 }
 
+// The merged row of a split item, f0 * O_0 + f1 * O_1 (the weights carry the
+// two halves' rescale to the common maximum and the 1 / l), converted and
+// stored; 32 columns of each half at a time.
+template <int DP, bool kBF16>
+__device__ __forceinline__ void store_row_merged(uint32_t tO0, uint32_t tO1, float f0, float f1, uint8_t* orow,
+                                                 bool row_ok, int D) {
+    auto emit = [&](int col, const uint32_t* a, const uint32_t* b, int n) {
+        for (int g = 0; g < n / 8; ++g) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int x = 8 * g + 2 * i;
+                w[i] = ptx::pack2<kBF16>(fmaf(__uint_as_float(a[x]), f0, __uint_as_float(b[x]) * f1),
+                                         fmaf(__uint_as_float(a[x + 1]), f0, __uint_as_float(b[x + 1]) * f1));
+            }
+            if (row_ok && col + 8 * g + 8 <= D) ptx::st_global_v4(orow + 2 * (col + 8 * g), w[0], w[1], w[2], w[3]);
+        }
+    };
+#pragma unroll
+    for (int c = 0; c + 32 <= DP; c += 32) {
+        uint32_t a[32], b[32];
+        ptx::tmem_ld32(tO0 + c, a);
+        ptx::tmem_ld32(tO1 + c, b);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) emit(c + 8 * g, a + 8 * g, b + 8 * g, 8);
+    }
+    if (DP % 32) {
+        constexpr int c = DP - 16;
+        uint32_t a[16], b[16];
+        ptx::tmem_ld16(tO0 + c, a);
+        ptx::tmem_ld16(tO1 + c, b);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 2; ++g) emit(c + 8 * g, a + 8 * g, b + 8 * g, 8);
+    }
+}
+
 // Zeros for this thread's output row (a query that sees no key).
 __device__ __forceinline__ void store_zero_row(uint8_t* orow, bool row_ok, int D) {
     if (!row_ok) return;
@@ -544,19 +611,23 @@ __device__ __forceinline__ Item item_of(const FwdParams& p, const SegTable<kVarl
         it.nk = p.Nk;
     }
     it.q0 = qg * (p.tiles_per_cta * kTileRows);
-    it.nt = (p.tiles_per_cta == 2 && it.q0 + kTileRows < it.n) ? 2 : 1;
+    it.nt = (p.split || (p.tiles_per_cta == 2 && it.q0 + kTileRows < it.n)) ? 2 : 1;
     return it;
 }
 
 // The CTA's k-th work item: looping CTAs take items blockIdx.x + k * gridDim.x.
 __device__ __forceinline__ int local_item(int k) { return (int)blockIdx.x + k * (int)gridDim.x; }
 
-// Key blocks an item runs over: its keys, and with the causal mask only up to
-// the last key its last query row sees (0 if no row sees any key).
+// Key blocks each tile of an item runs over: its keys, and with the causal
+// mask only up to the last key its last query row sees (0 if no row sees any
+// key).  A split item's two halves take ceil(blocks / 2) each (the upper half
+// starts at that block; with an odd count its last block lies past the keys
+// and is masked whole).
 __device__ __forceinline__ int item_kblocks(const FwdParams& p, const Item& it) {
     int keys = it.nk;
     if (p.causal) keys = max(0, min(keys, min(it.q0 + it.nt * kTileRows, it.n) + p.causal_off));
-    return (keys + kBlockKeys - 1) / kBlockKeys;
+    const int blocks = (keys + kBlockKeys - 1) / kBlockKeys;
+    return p.split ? (blocks + 1) / 2 : blocks;
 }
 
 // ---------------------------------------------------------------- roles
@@ -567,8 +638,11 @@ __device__ __forceinline__ int item_kblocks(const FwdParams& p, const Item& it) 
 // (slot = entry % kStages, refilled once the MMAs that read the previous
 // occupant have completed).  Before returning it waits (bounded) for every
 // copy it started, so that no copy lands after an abort has ended the CTA.
-// Every item of the CTA has nkb key blocks.
-template <int DP, int NQ, int kStages, bool kLoop, bool kVarlen>
+// Every item of the CTA has nkb key blocks per tile.  kSplit: both tiles are
+// the item's one query tile (its Q is loaded into both buffers), tile t runs
+// over key blocks t*nkb + j, and every unit has its own K/V pair: the ring
+// takes K_j, V_j, K_{nkb+j}, V_{nkb+j} for each j.
+template <int DP, int NQ, int kStages, bool kLoop, bool kVarlen, bool kSplit = false>
 __device__ __forceinline__ void produce(const FwdParams& p, const SegTable<kVarlen>& seg, uint32_t sQ, uint32_t sKV,
                                         uint32_t sBar, volatile int* abort_flag, int n_my, int T, int nkb,
                                         uint64_t tmo) {
@@ -599,12 +673,13 @@ __device__ __forceinline__ void produce(const FwdParams& p, const SegTable<kVarl
             for (int c = 0; c < NCH; ++c)
                 ptx::tma_load_4d(sQ + (qb * kTilesPerCta + t) * TILE + 256 * chunk_col(DP, c),
                                  &p.maps[0][width_class(chunk_width(DP, c))], chunk_col(DP, c), it.h,
-                                 it.tok0 + it.q0 + t * kTileRows, it.b, bar(kBarQFull + 2 * qb + t));
+                                 it.tok0 + it.q0 + (kSplit ? 0 : t * kTileRows), it.b, bar(kBarQFull + 2 * qb + t));
             if (t == 0) q_last0 = k;
             else q_last1 = k;
         }
 
-        for (int j = 0; j < nkb && ok; ++j) {
+        for (int u = 0; u < nkb * (kSplit ? T : 1) && ok; ++u) {
+            const int j = kSplit ? (u >> 1) + (u & 1) * nkb : u;  // key block of this K/V pair
             for (int kv = 0; kv < 2; ++kv, ++r) {
                 const int slot = r % kStages;
                 const uint32_t phase = (uint32_t)(r / kStages) & 1u;
@@ -722,16 +797,25 @@ __device__ __forceinline__ void issue_pv(uint32_t d, uint32_t a, uint32_t v_tile
 // kVarlen: a ragged batch (tokens of several images packed along the N axis
 // of a B = 1 tensor, described by `seg`); each work item attends within its
 // own segment.  Ragged batches run one item per CTA.
-template <int DP, bool kBF16, bool kLoop, bool kVarlen>
+// kSplit (one item per CTA): the item is one query tile, and the two softmax
+// warpgroups take the lower and upper halves of its key blocks with their
+// own running (m, l, O); at the end the upper half hands (m, l) over shared
+// memory to the lower, which reads the upper O out of TMEM and writes
+//   O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m)),
+// m = max(m_0, m_1): the same online-softmax merge the key blocks of one half
+// already go through, applied once more.  This halves the serial chain of a
+// CTA when the items are too few to fill the SMs with two tiles each.
+template <int DP, bool kBF16, bool kLoop, bool kVarlen, bool kSplit = false>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p,
                                                           const __grid_constant__ SegTable<kVarlen> seg) {
     constexpr int TILE = tile_bytes(DP);
     constexpr int NCH = chunk_count(DP);
     static_assert(DP % 16 == 0 && DP >= 16 && DP <= 128, "head dim padding");
     static_assert(!(kLoop && kVarlen), "ragged batches run one work item per CTA");
+    static_assert(!kSplit || (!kLoop && !kVarlen), "split items run one per CTA, dense layout");
 
     constexpr int NQ = q_buffers(DP, kLoop);
-    constexpr int kStages = kv_stages(DP);
+    constexpr int kStages = kv_stages(DP, kSplit);
     constexpr int kVSlots = kStages / 2;  // V_g sits in V slot g % kVSlots, its use g / kVSlots
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = ptx::smem_u32(smem_raw);
@@ -743,6 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     uint32_t* const tmem_holder =
         reinterpret_cast<uint32_t*>(base_ptr + (NQ * kTilesPerCta + kStages) * TILE + kNumBars * 8);
     volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    float* const merge_ml = reinterpret_cast<float*>(tmem_holder + 4);  // [2][128] (m, l) of the upper half
     auto bar = [&](int i) -> uint32_t { return sBar + 8u * (uint32_t)i; };
 
     const int warp = threadIdx.x >> 5;
@@ -779,6 +864,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             for (int vs = t; vs < kMaxStages / 2; vs += 2) ptx::mbar_init(bar(kBarVReady + vs), 2 * 32);
         }
         ptx::mbar_init(bar(kBarDrain), 1);
+        ptx::mbar_init(bar(kBarMerge), 4 * 32);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -798,7 +884,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0)
-            produce<DP, NQ, kStages, kLoop, kVarlen>(p, seg, sQ, sKV, sBar, abort_flag, n_my, T, nkb, tmo);
+            produce<DP, NQ, kStages, kLoop, kVarlen, kSplit>(p, seg, sQ, sKV, sBar, abort_flag, n_my, T, nkb, tmo);
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -826,6 +912,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             struct Cursor {
                 int t, j, k, g, buf;  // tile, block, item (local index), block count g = k*nkb + j, S buffer
             };
+            // The K/V pair a unit reads: block g's, shared by its tiles -- or, for a
+            // split item, the unit's own (its tiles read different key blocks).
+            auto kv_pair = [&](const Cursor& c) -> int { return kSplit ? T * c.g + c.t : c.g; };
             auto advance = [&](Cursor& c) {
                 if (++c.t == T) {
                     c.t = 0;
@@ -846,14 +935,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                         return false;
                     ptx::tc_fence_after();
                 }
-                if (c.t == 0) {
-                    if (!wait_warp(bar(kBarKvFull + kv_slot(2 * c.g)), kv_parity(2 * c.g), abort_flag, tmo, 3))
+                const int e = kv_pair(c);
+                if (kSplit || c.t == 0) {
+                    if (!wait_warp(bar(kBarKvFull + kv_slot(2 * e)), kv_parity(2 * e), abort_flag, tmo, 3))
                         return false;
                     ptx::tc_fence_after();
                 }
-                mma_s(qb * kTilesPerCta + c.t, kv_slot(2 * c.g), c.buf);
+                mma_s(qb * kTilesPerCta + c.t, kv_slot(2 * e), c.buf);
                 ptx::mma_commit_w(bar(kBarSFull + c.buf), leader);
-                if (c.t == T - 1) ptx::mma_commit_w(bar(kBarKvEmpty + kv_slot(2 * c.g)), leader);
+                if (kSplit || c.t == T - 1) ptx::mma_commit_w(bar(kBarKvEmpty + kv_slot(2 * e)), leader);
                 if (kLoop && c.j == nkb - 1) ptx::mma_commit_w(bar(kBarQEmpty + 2 * qb + c.t), leader);
                 return true;
             };
@@ -861,13 +951,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             // bf16 inputs converted to f16) and released after its last.  V-ready
             // is per V slot: the converter reaches the slot's next block only after
             // it lands there, which needs the last P.V of this one, so the parity is
-            // unambiguous.
+            // unambiguous.  (K/V pair e: K in ring entry 2e, V in 2e + 1.)
             auto issue_pv = [&](const Cursor& c) -> bool {
                 const int t = c.t, j = c.j, g = c.g;
-                if (t == 0 &&
-                    !(kBF16 ? wait_warp(bar(kBarVReady + g % kVSlots), (uint32_t)(g / kVSlots) & 1u, abort_flag,
+                const int e = kv_pair(c);
+                if ((kSplit || t == 0) &&
+                    !(kBF16 ? wait_warp(bar(kBarVReady + e % kVSlots), (uint32_t)(e / kVSlots) & 1u, abort_flag,
                                         tmo, 4)
-                            : wait_warp(bar(kBarKvFull + kv_slot(2 * g + 1)), kv_parity(2 * g + 1), abort_flag,
+                            : wait_warp(bar(kBarKvFull + kv_slot(2 * e + 1)), kv_parity(2 * e + 1), abort_flag,
                                        tmo, 4)))
                     return false;
                 // the first product of an item overwrites O_t: the previous item's
@@ -878,9 +969,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 if (!wait_warp(bar(kBarPFull + 2 * t + (g & 1)), (uint32_t)(g >> 1) & 1u, abort_flag, tmo, 5))
                     return false;
                 ptx::tc_fence_after();
-                mma_pv(t, kv_slot(2 * g + 1), c.buf, j > 0);
+                mma_pv(t, kv_slot(2 * e + 1), c.buf, j > 0);
                 if (track_pv) ptx::mma_commit_w(bar(kBarOReady + t), leader);
-                if (t == T - 1) ptx::mma_commit_w(bar(kBarKvEmpty + kv_slot(2 * g + 1)), leader);
+                if (kSplit || t == T - 1) ptx::mma_commit_w(bar(kBarKvEmpty + kv_slot(2 * e + 1)), leader);
                 if (j == nkb - 1) ptx::mma_commit_w(bar(kBarOFull + t), leader);
                 return true;
             };
@@ -911,8 +1002,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         __syncwarp();
     } else if (kBF16) {
         // ------------------------------------------------------------ V converter (bf16)
-        convert_v_blocks<TILE, kStages>(base_ptr + (sKV - base), sBar, kBarVReady, abort_flag, n_my * nkb, tmo,
-                                        (int)threadIdx.x - kConvWarp * 32);
+        convert_v_blocks<TILE, kStages>(base_ptr + (sKV - base), sBar, kBarVReady, abort_flag,
+                                        n_my * nkb * (kSplit ? T : 1), tmo, (int)threadIdx.x - kConvWarp * 32);
     }
     } else {
         ptx::setmaxnreg_inc<kSoftmaxRegs>();
@@ -941,11 +1032,38 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 if (kb > 0 && !wait_warp(bar(kBarOFull + t), (uint32_t)phase & 1u, abort_flag, tmo, 8)) return false;
                 ptx::tc_fence_after();
                 const Item it = my_item(k);
-                const int row = it.q0 + t * kTileRows + wq * 32 + lane;
+                const int row = it.q0 + (kSplit ? 0 : t * kTileRows) + wq * 32 + lane;
                 uint8_t* orow =
                     reinterpret_cast<uint8_t*>(p.out) +
                     ((((size_t)it.b * p.N + (size_t)it.tok0 + (size_t)min(row, it.n - 1)) * p.H + it.h) * p.D) * 2;
                 const uint32_t o_empty = kLoop ? bar(kBarOEmpty + t) : 0u;
+                if constexpr (kSplit) {
+                    // the upper half hands its (m, l) over; the lower half waits for
+                    // both halves' last P.V and that hand-over, then merges
+                    const int rl = wq * 32 + lane;
+                    if (t == 1) {
+                        merge_ml[rl] = m_used;
+                        merge_ml[kTileRows + rl] = l;
+                        ptx::mbar_arrive(bar(kBarMerge));
+                        return true;
+                    }
+                    if (!wait_warp(bar(kBarOFull + 1), 0u, abort_flag, tmo, 15) ||
+                        !wait_warp(bar(kBarMerge), 0u, abort_flag, tmo, 16))
+                        return false;
+                    ptx::tc_fence_after();
+                    const float m1 = merge_ml[rl], l1 = merge_ml[kTileRows + rl];
+                    const float m = fmaxf(m_used, m1);
+                    const float a0 = m_used == -INFINITY ? 0.f : ptx::ex2(m_used - m);
+                    const float a1 = m1 == -INFINITY ? 0.f : ptx::ex2(m1 - m);
+                    const float lm = l * a0 + l1 * a1;
+                    const float inv = lm > 0.f ? 1.f / lm : 0.f;
+                    store_row_merged<DP, kBF16>(tO, tO + (uint32_t)o_cols(DP), a0 * inv, a1 * inv, orow, row < it.n,
+                                                p.D);
+                    if (p.lse != nullptr && row < it.n)
+                        p.lse[((size_t)it.b * p.H + it.h) * p.N + it.tok0 + row] =
+                            lm > 0.f ? (m + log2f(lm)) * 0.6931471805599453f : -INFINITY;
+                    return true;
+                }
                 // a row that saw no key (causal, more queries than keys) is 0
                 if (kb > 0) {
                     store_row<DP, kBF16>(tO, l > 0.f ? 1.f / l : 0.f, orow, row < it.n, p.D, o_empty);
@@ -964,7 +1082,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             for (int k = 0; k < n_my && ok; ++k) {
             const Item it = my_item(k);
             const int kb = nkb;
-            const int row = it.q0 + t * kTileRows + wq * 32 + lane;
+            const int row = it.q0 + (kSplit ? 0 : t * kTileRows) + wq * 32 + lane;
+            const int kb0 = kSplit ? t * kb : 0;  // this tile's first key block
             float m_used = -INFINITY;
             float l = 0.f;
             for (int j = 0; j < kb; ++j, ++g) {
@@ -995,8 +1114,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 // keys of this block the row sees: the ragged tail, and with the
                 // causal mask the row's own limit (<= 0: none); "partial" is decided
                 // warp-wide because the exp path holds warp-collective TMEM stores
-                int valid = min(kBlockKeys, it.nk - j * kBlockKeys);
-                if (p.causal) valid = min(valid, row + p.causal_off + 1 - j * kBlockKeys);
+                int valid = min(kBlockKeys, it.nk - (kb0 + j) * kBlockKeys);
+                if (p.causal) valid = min(valid, row + p.causal_off + 1 - (kb0 + j) * kBlockKeys);
                 const bool partial = __any_sync(0xffffffffu, valid < kBlockKeys);
                 const float ext = partial ? (neg ? row_extreme<true, true>(s, valid)
                                                  : row_extreme<true, false>(s, valid))

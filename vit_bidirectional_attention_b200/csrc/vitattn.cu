@@ -267,8 +267,9 @@ bool encode_map(CUtensorMap* m, const void* ptr, int dtype, int64_t B, int64_t N
 
 // ---------------------------------------------------------------- dispatch
 
-// Kernel modes: one work item per CTA, CTAs looping over items, ragged batch.
-enum Mode { kModeItem = 0, kModeLoop = 1, kModeVarlen = 2, kNumModes = 3 };
+// Kernel modes: one work item per CTA, CTAs looping over items, ragged batch,
+// one split item (a query tile's key blocks in two halves) per CTA.
+enum Mode { kModeItem = 0, kModeLoop = 1, kModeVarlen = 2, kModeSplit = 3, kNumModes = 4 };
 
 template <int DP>
 const void* kernel_of(bool bf, Mode mode) {
@@ -279,6 +280,9 @@ const void* kernel_of(bool bf, Mode mode) {
         case kModeVarlen:
             return bf ? reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, true, false, true>)
                       : reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, false, false, true>);
+        case kModeSplit:
+            return bf ? reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, true, false, false, true>)
+                      : reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, false, false, false, true>);
         default:
             return bf ? reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, true, false, false>)
                       : reinterpret_cast<const void*>(vitattn::fwd_kernel<DP, false, false, false>);
@@ -368,7 +372,7 @@ int ensure_smem(int dp, int dtype, Mode mode, const void* fn) {
     bool& done = g_dev[dev].smem_set[dp / 16][dtype][mode];
     if (!done) {
         e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 vitattn::smem_bytes(dp, mode == kModeLoop));
+                                 vitattn::smem_bytes(dp, mode == kModeLoop, mode == kModeSplit));
         if (e != cudaSuccess) return cuda_fail(e);
         done = true;
     }
@@ -419,7 +423,7 @@ int run_kernel(int dp, int dtype, Mode mode, unsigned grid, FwdParams* prm, Seg*
     if (rc) return rc;
     void* args[2] = {prm, seg};
     cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(vitattn::kThreads), args,
-                                     (size_t)vitattn::smem_bytes(dp, mode == kModeLoop), stream);
+                                     (size_t)vitattn::smem_bytes(dp, mode == kModeLoop, mode == kModeSplit), stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return VITATTN_OK;
 }
@@ -477,9 +481,17 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     if (uniform && prm.n_items > num_sms && prm.n_kblocks <= 32) grid = (unsigned)num_sms;
     if (uniform && (flags & vitattn::kFlagTinyGrid) && grid > 3u) grid = 3u;
     const bool loop = grid < (unsigned)prm.n_items;
+    // One query tile per item (two would leave SMs idle) and one CTA per
+    // item: the tile's key blocks are split over the two softmax warpgroups,
+    // so that the CTA's serial chain is half as long and both warpgroups
+    // work (the unmasked case with at least four key blocks).
+    const int split_from = (flags & vitattn::kFlagSplitFromTwo) ? 2 : 4;
+    prm.split = !loop && !prm.causal && prm.tiles_per_cta == 1 && prm.n_kblocks >= split_from &&
+                !(flags & vitattn::kFlagNoSplit);
 
     SegDense seg{0};
-    return run_kernel(dp, dtype, loop ? kModeLoop : kModeItem, grid, &prm, &seg, stream);
+    return run_kernel(dp, dtype, loop ? kModeLoop : (prm.split ? kModeSplit : kModeItem), grid, &prm, &seg,
+                      stream);
 }
 
 // Ragged batch: one CTA per work item (segment, head, group of query tiles).
