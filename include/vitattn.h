@@ -375,18 +375,21 @@ VITATTN_API int vitattn_check_args_qk_norm_rope(const void* qkv, const float* co
  * `flash_attn_gpu`: upload the inputs, run the device entry, read the
  * output back).  Here the caller supplies the device staging buffers, so
  * the library still allocates no memory.
- *   The batch is split into up to 8 groups of whole images; group c's
- *   inputs are copied in while the kernel of group c-1 runs and the output
- *   of group c-2 is copied out.  The copies run on two streams the library
- *   keeps per host thread and device (created on the first call); the
- *   kernels run on `stream`.  The copies start after the work already
+ *   The work is cut into up to 8 groups: runs of whole images when B >= 8,
+ *   otherwise groups of heads of one image (rows of at least 1 KB of each
+ *   token's heads, copied with 2-D copies; heads are independent).  Group
+ *   c's inputs are copied in while the kernel of group c-1 runs and the
+ *   output of group c-2 is copied out.  The copies run on two streams the
+ *   library keeps per host thread and device (created on the first call);
+ *   the kernels run on `stream`.  The copies start after the work already
  *   enqueued on `stream`, and work enqueued on `stream` after this call (or
  *   a synchronisation of `stream`) comes after the last output copy, so the
  *   caller synchronises `stream` before reading hout, as with one stream.
  *   Host buffers should be pinned (cudaHostAlloc / cudaHostRegister) for the
  *   copies to overlap; dq, dk, dv, dout are caller-owned device staging with
  *   the requirements of vitattn_forward.  All eight pointers are required.
- *   Launches one kernel per group.
+ *   Launches one kernel per group.  A group of heads writes its part of the
+ *   output rows; the other heads' columns of dout are left to their groups.
  */
 VITATTN_API int vitattn_forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq,
                          void* dk, void* dv, void* dout, int64_t B, int64_t N, int64_t H,

@@ -7,6 +7,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 from vit_bidirectional_attention_b200 import vitattn
@@ -312,3 +313,26 @@ def test_qk_rope_checks_need_no_v_and_refuse_aliasing():
     assert vitattn.check_args_qk_rope(qkv, cs, sn, qkv + 64, k, T, H, D, vitattn.BF16) == -6  # q inside qkv
     assert vitattn.check_args_qk_rope(qkv, cs, sn, 0, k, T, H, D, vitattn.BF16) == -1
     assert vitattn.check_args_qk_rope(qkv, cs, sn, q, k, T, H, 72, 7) == -4
+
+
+@pytest.mark.parametrize("B,H,D", [(1, 16, 64), (2, 16, 128), (3, 12, 80), (1, 1, 64), (1, 3, 16), (7, 5, 32),
+                                   (16, 4, 64), (32, 16, 64), (9, 4, 64), (1, 40, 128), (4, 2, 128)])
+def test_host_plan_covers_every_image_and_head_once(B, H, D):
+    """The host-buffer entry's cut of a batch: every (image, head) in exactly
+    one group, at most 8 groups, and when heads are cut each copied row of
+    a group is at least 1 KB wide."""
+    per_chunk, G, n = vitattn.host_plan(B, H, D)
+    assert 1 <= n <= 8
+    seen = np.zeros((B, H), dtype=int)
+    for c in range(n):
+        if G > 1:
+            b0, nb, h0 = c // G, 1, (c % G) * H // G
+            nh = (c % G + 1) * H // G - h0
+            assert nh * D * 2 >= 1024
+        else:
+            b0, nb, h0, nh = c * per_chunk, min(per_chunk, B - c * per_chunk), 0, H
+        assert nb >= 1 and nh >= 1
+        seen[b0:b0 + nb, h0:h0 + nh] += 1
+    assert np.all(seen == 1)
+    if B >= 8:
+        assert G == 1  # whole images when there are enough of them

@@ -290,6 +290,32 @@ def test_host_buffer_entry_multi_group(cuda_device, B):
     assert np.array_equal(from_dev(hout, synth.BF16), first)
 
 
+@pytest.mark.parametrize("B,N,H,D", [(1, 300, 16, 64), (2, 700, 16, 128), (3, 257, 15, 80)])
+def test_host_buffer_entry_head_groups(cuda_device, B, N, H, D):
+    # fewer images than groups: each image travels as groups of heads (2-D
+    # copies of the heads' columns, token-strided attention and output);
+    # the output must match the oracle and, within the tolerance, the device
+    # entry, and every head column of every row must be written
+    import torch
+
+    per_chunk, G, n = vitattn.host_plan(B, H, D)
+    assert G > 1 and n == B * G
+    q, k, v = synth.random_qkv(B, N, H, D, synth.BF16, seed=41 + N + H)
+    hosts = [torch.from_numpy(x.view(np.int16).copy()).view(torch.bfloat16).pin_memory() for x in (q, k, v)]
+    hout = torch.full_like(hosts[0], float("nan")).pin_memory()
+    dq, dk, dv, dout = (torch.empty(q.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    s = torch.cuda.Stream()
+    args = [h.data_ptr() for h in hosts] + [hout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                            dout.data_ptr(), B, N, H, D, 1.0 / math.sqrt(D), synth.BF16, s.cuda_stream]
+    assert vitattn.forward_host_ptr(*args) == 0
+    s.synchronize()
+    got = from_dev(hout, synth.BF16)
+    assert np.all(np.isfinite(got))
+    assert_close(got, oracle.attention(q, k, v, 1.0 / math.sqrt(D), synth.BF16), f"head groups {B}x{N}x{H}x{D}")
+    dev = vitattn.forward(dq, dk, dv, scale=1.0 / math.sqrt(D), checked=True)
+    assert_close(got, from_dev(dev, synth.BF16), "host vs device entry")
+
+
 def test_pointers_of_host_memory_are_refused(cuda_device):
     # a plain (unregistered) host pointer passed as device memory is refused
     # before anything is enqueued, instead of reaching a tensor map

@@ -227,6 +227,7 @@ struct SegTable<true> {
 struct alignas(64) FwdParams {
     CUtensorMap maps[3][3];  // [q, k, v][width class 64 / 32 / 16]
     void* out;
+    long long out_ts;   // elements between consecutive tokens of out (H * D when dense)
     int B, N, H, D;
     int tiles_per_cta;  // query tiles a work item owns: 2, or 1 when 2 would leave SMs idle
     int n_qgroups;      // ceil(N / (128 * tiles_per_cta)): work items per (b, h) (dense layout)
@@ -1033,9 +1034,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                 ptx::tc_fence_after();
                 const Item it = my_item(k);
                 const int row = it.q0 + (kSplit ? 0 : t * kTileRows) + wq * 32 + lane;
-                uint8_t* orow =
-                    reinterpret_cast<uint8_t*>(p.out) +
-                    ((((size_t)it.b * p.N + (size_t)it.tok0 + (size_t)min(row, it.n - 1)) * p.H + it.h) * p.D) * 2;
+                uint8_t* orow = reinterpret_cast<uint8_t*>(p.out) +
+                                (((size_t)it.b * p.N + (size_t)it.tok0 + (size_t)min(row, it.n - 1)) *
+                                     (size_t)p.out_ts + (size_t)it.h * p.D) * 2;
                 const uint32_t o_empty = kLoop ? bar(kBarOEmpty + t) : 0u;
                 if constexpr (kSplit) {
                     // the upper half hands its (m, l) over; the lower half waits for

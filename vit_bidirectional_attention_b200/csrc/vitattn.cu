@@ -113,11 +113,12 @@ int check_args_gqa(const void* q, const void* k, const void* v, const void* out,
 
 // Token-strided inputs: element (b, i, h, d) of x at x + ((b*N + i)*ts_x + h*D + d)
 // for x = q, k, v (ts_x elements between consecutive tokens, >= H*D, a multiple
-// of 8 so that every token row starts on 16 bytes); out dense [B, N, H, D].
-// The inputs may overlap one another (views of one packed projection); out
-// must not overlap any of them.
+// of 8 so that every token row starts on 16 bytes); out dense [B, N, H, D], or
+// (internally, for head groups of the host-buffer entry) token-strided by
+// out_ts likewise.  The inputs may overlap one another (views of one packed
+// projection); out must not overlap any of them.
 int check_args_strided(const void* q, const void* k, const void* v, const void* out, int64_t B, int64_t N,
-                       int64_t H, int64_t D, const int64_t ts[3], float scale, int dtype) {
+                       int64_t H, int64_t D, const int64_t ts[3], float scale, int dtype, int64_t out_ts = 0) {
     if (!q || !k || !v || !out) return VITATTN_ERR_NULL;
     if (B < 1 || N < 1 || H < 1 || D < 1) return VITATTN_ERR_DIM;
     if (D < 16 || D > 128 || D % 8 != 0) return VITATTN_ERR_HEADDIM;
@@ -140,7 +141,11 @@ int check_args_strided(const void* q, const void* k, const void* v, const void* 
     const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                            reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out)) & 15u;
     if (mis) return VITATTN_ERR_ALIGN;
-    const uint64_t out_bytes = out_bytes_batch * (uint64_t)B;
+    if (out_ts != 0 && (out_ts < (int64_t)row || out_ts % 8 != 0 ||
+                        (uint64_t)N * (uint64_t)out_ts * 2u >= (1ull << 40)))
+        return VITATTN_ERR_DIM;
+    const uint64_t out_bytes = out_ts == 0 ? out_bytes_batch * (uint64_t)B
+                                           : ((uint64_t)B * (uint64_t)N - 1u) * (uint64_t)out_ts * 2u + row * 2u;
     if (overlaps2(out, out_bytes, q, extent[0]) || overlaps2(out, out_bytes, k, extent[1]) ||
         overlaps2(out, out_bytes, v, extent[2]))
         return VITATTN_ERR_ALIAS;
@@ -404,6 +409,7 @@ int fill_common(FwdParams* prm, const void* q, const void* k, const void* v, voi
     prm->kv_group = (int)(H / Hkv);
     prm->Nk = (int)Nk;
     prm->out = out;
+    prm->out_ts = (long long)(H * D);
     prm->B = (int)B;
     prm->N = (int)N;
     prm->H = (int)H;
@@ -434,12 +440,13 @@ struct Ext {
     int causal = 0;       // aligned causal mask
     float* lse = nullptr; // optional [B, H, N] log-sum-exp output
     const int64_t* ts = nullptr;  // token strides of q, k, v in elements; nullptr: dense
+    int64_t out_ts = 0;           // token stride of out in elements (with ts only); 0: dense
 };
 
 int launch(const void* q, const void* k, const void* v, void* out, int64_t B, int64_t N,
            int64_t H, int64_t D, float scale, int dtype, cudaStream_t stream, int flags, int64_t Hkv = 0,
            const Ext& ext = Ext()) {
-    int rc = ext.ts   ? check_args_strided(q, k, v, out, B, N, H, D, ext.ts, scale, dtype)
+    int rc = ext.ts   ? check_args_strided(q, k, v, out, B, N, H, D, ext.ts, scale, dtype, ext.out_ts)
              : ext.Nk ? check_args_ext(q, k, v, out, ext.lse, B, N, ext.Nk, H, D, scale, dtype)
              : Hkv    ? check_args_gqa(q, k, v, out, B, N, H, Hkv, D, scale, dtype)
                       : check_args(q, k, v, out, B, N, H, D, scale, dtype);
@@ -455,6 +462,7 @@ int launch(const void* q, const void* k, const void* v, void* out, int64_t B, in
     FwdParams prm;
     rc = fill_common(&prm, q, k, v, out, B, N, H, D, scale, dtype, flags, Hkv, Nk, ext.ts);
     if (rc) return rc;
+    if (ext.out_ts) prm.out_ts = (long long)ext.out_ts;
     prm.causal = ext.causal ? 1 : 0;
     prm.causal_off = (int)(Nk - N);
     prm.lse = ext.lse;
@@ -645,12 +653,18 @@ int forward_varlen_checked(const void* q, const void* k, const void* v, void* ou
 
 // ---------------------------------------------------------------- host-buffer entry
 
-// The host-buffer entry splits the batch into up to kHostChunks groups of
-// whole images so that copies and kernels overlap: the inputs of group c+1
-// travel host -> device while the kernel of group c runs and the output of
-// group c-1 travels back.  Two copy streams per (host thread, device) carry
-// the two directions; the kernels run on the caller's stream.
+// The host-buffer entry cuts the work into up to kHostChunks groups so that
+// copies and kernels overlap: the inputs of group c+1 travel host -> device
+// while the kernel of group c runs and the output of group c-1 travels back.
+// A group is a run of whole images when the batch has at least kHostChunks
+// of them; otherwise each image is cut into groups of heads (every head of
+// a token is independent), copied as 2-D copies of the heads' columns
+// (rows of at least kMinCopyRow bytes, so the copy engines stay efficient)
+// and run through the token-strided attention with a token-strided output.
+// Two copy streams per (host thread, device) carry the two directions; the
+// kernels run on the caller's stream.
 constexpr int kHostChunks = 8;
+constexpr int64_t kMinCopyRow = 1024;
 
 struct HostPipe {
     bool ready = false;
@@ -678,6 +692,35 @@ int host_pipe(int dev, HostPipe** out) {
     return VITATTN_OK;
 }
 
+// How the host-buffer entry cuts [B, N, H, D]: `per_chunk` images per group
+// when heads are not cut (groups_per_image == 1), else one image per group
+// and its heads in groups_per_image near-equal parts: part g is heads
+// g*H/G .. (g+1)*H/G - 1 (G = groups_per_image, integer division), each at
+// least kMinCopyRow bytes of a token wide.
+struct HostPlan {
+    int64_t per_chunk;
+    int groups_per_image, nchunks;
+};
+
+HostPlan host_plan(int64_t B, int64_t H, int64_t D) {
+    HostPlan pl{};
+    pl.groups_per_image = 1;
+    if (B < kHostChunks && H > 1) {
+        const int64_t want = (kHostChunks + B - 1) / B;              // groups per image wanted
+        const int64_t min_hc = (kMinCopyRow + 2 * D - 1) / (2 * D);  // heads per copy row at least
+        const int64_t g = std::min<int64_t>(std::min<int64_t>(want, H / min_hc), kHostChunks / B);
+        if (g > 1) pl.groups_per_image = (int)g;
+    }
+    if (pl.groups_per_image > 1) {
+        pl.per_chunk = 1;
+        pl.nchunks = (int)(B * pl.groups_per_image);
+    } else {
+        pl.per_chunk = (B + kHostChunks - 1) / kHostChunks;
+        pl.nchunks = (int)((B + pl.per_chunk - 1) / pl.per_chunk);
+    }
+    return pl;
+}
+
 int forward_host(const void* hq, const void* hk, const void* hv, void* hout, void* dq, void* dk, void* dv,
                  void* dout, int64_t B, int64_t N, int64_t H, int64_t D, float scale, int dtype,
                  cudaStream_t s) {
@@ -696,40 +739,55 @@ int forward_host(const void* hq, const void* hk, const void* hv, void* hout, voi
     rc = host_pipe(dev, &hp);
     if (rc) return rc;
 
-    const int64_t per_chunk = (B + kHostChunks - 1) / kHostChunks;  // images per group
-    const int nchunks = (int)((B + per_chunk - 1) / per_chunk);
-    const size_t image_bytes = (size_t)N * (size_t)H * (size_t)D * 2u;
+    const HostPlan pl = host_plan(B, H, D);
+    const size_t token_bytes = (size_t)H * (size_t)D * 2u;
+    const size_t image_bytes = (size_t)N * token_bytes;
     const void* hsrc[3] = {hq, hk, hv};
     uint8_t* ddst[3] = {static_cast<uint8_t*>(dq), static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv)};
+    const int64_t ts[3] = {H * D, H * D, H * D};
     // the copies start once the caller's earlier work on `s` is done (it may still read dq..dout)
     e = cudaEventRecord(hp->start, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->h2d, hp->start, 0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->d2h, hp->start, 0);
     if (e != cudaSuccess) return cuda_fail(e);
-    for (int c = 0; c < nchunks; ++c) {
-        const int64_t b0 = (int64_t)c * per_chunk;
-        const int64_t nb = std::min<int64_t>(per_chunk, B - b0);
-        const size_t off = (size_t)b0 * image_bytes, bytes = (size_t)nb * image_bytes;
+    for (int c = 0; c < pl.nchunks; ++c) {
+        // group c: images b0 .. b0 + nb - 1, heads h0 .. h0 + nh - 1
+        const int G = pl.groups_per_image;
+        const int64_t b0 = (G > 1) ? c / G : (int64_t)c * pl.per_chunk;
+        const int64_t nb = (G > 1) ? 1 : std::min<int64_t>(pl.per_chunk, B - b0);
+        const int64_t h0 = (G > 1) ? (c % G) * H / G : 0;
+        const int64_t nh = (G > 1) ? (c % G + 1) * H / G - h0 : H;
+        const size_t off = (size_t)b0 * image_bytes + (size_t)h0 * (size_t)D * 2u;
+        const size_t width = (size_t)nh * (size_t)D * 2u;  // bytes of one token's heads in the group
+        const size_t rows = (size_t)nb * (size_t)N;
+        auto copy = [&](void* dst, const void* src, cudaMemcpyKind kind, cudaStream_t st) -> cudaError_t {
+            if (nh == H) return cudaMemcpyAsync(dst, src, rows * width, kind, st);
+            return cudaMemcpy2DAsync(dst, token_bytes, src, token_bytes, width, rows, kind, st);
+        };
         for (int i = 0; i < 3 && e == cudaSuccess; ++i)
-            e = cudaMemcpyAsync(ddst[i] + off, static_cast<const uint8_t*>(hsrc[i]) + off, bytes,
-                                cudaMemcpyHostToDevice, hp->h2d);
+            e = copy(ddst[i] + off, static_cast<const uint8_t*>(hsrc[i]) + off, cudaMemcpyHostToDevice, hp->h2d);
         if (e == cudaSuccess) e = cudaEventRecord(hp->in[c], hp->h2d);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hp->in[c], 0);
         if (e != cudaSuccess) return cuda_fail(e);
-        rc = launch(ddst[0] + off, ddst[1] + off, ddst[2] + off, static_cast<uint8_t*>(dout) + off, nb, N, H, D,
-                    scale, dtype, s, 0);
+        uint8_t* o = static_cast<uint8_t*>(dout) + off;
+        if (nh == H) {
+            rc = launch(ddst[0] + off, ddst[1] + off, ddst[2] + off, o, nb, N, H, D, scale, dtype, s, 0);
+        } else {
+            Ext ext;
+            ext.ts = ts;
+            ext.out_ts = H * D;
+            rc = launch(ddst[0] + off, ddst[1] + off, ddst[2] + off, o, nb, N, nh, D, scale, dtype, s, 0, 0, ext);
+        }
         if (rc) return rc;
         e = cudaEventRecord(hp->ran[c], s);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(hp->d2h, hp->ran[c], 0);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(static_cast<uint8_t*>(hout) + off, static_cast<const uint8_t*>(dout) + off, bytes,
-                                cudaMemcpyDeviceToHost, hp->d2h);
+        if (e == cudaSuccess) e = copy(static_cast<uint8_t*>(hout) + off, o, cudaMemcpyDeviceToHost, hp->d2h);
         if (e == cudaSuccess) e = cudaEventRecord(hp->out[c], hp->d2h);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     // work the caller enqueues on `s` afterwards (or a synchronisation of `s`) follows the last
     // output copy; the copy stream runs in order, so that covers every group
-    e = cudaStreamWaitEvent(s, hp->out[nchunks - 1], 0);
+    e = cudaStreamWaitEvent(s, hp->out[pl.nchunks - 1], 0);
     if (e != cudaSuccess) return cuda_fail(e);
     return VITATTN_OK;
 }
@@ -972,5 +1030,17 @@ int vitattn_last_cuda_error(void) { return t_last_cuda_error; }
 int vitattn_version(void) { return kVersion; }
 
 int vitattn_launches_per_call(void) { return 1; }
+
+// Test hook, deliberately absent from the public header: how the host-buffer
+// entry cuts a batch (out[0] images per group, out[1] groups per image, 1
+// when heads are not cut, out[2] groups).  No CUDA call.
+VITATTN_API int vitattn_test_host_plan(int64_t B, int64_t H, int64_t D, int64_t* out) {
+    if (!out || B < 1 || H < 1 || D < 1) return VITATTN_ERR_DIM;
+    const HostPlan pl = host_plan(B, H, D);
+    out[0] = pl.per_chunk;
+    out[1] = pl.groups_per_image;
+    out[2] = pl.nchunks;
+    return VITATTN_OK;
+}
 
 }  // extern "C"

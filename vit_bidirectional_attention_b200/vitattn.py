@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
         qk_norm_rope = [p, p, p, p, p, f32, p, p, i64, i64, i64, i32]
         L.vitattn_qk_norm_rope.argtypes = qk_norm_rope + [p]
         L.vitattn_check_args_qk_norm_rope.argtypes = qk_norm_rope
+        L.vitattn_test_host_plan.argtypes = [i64, i64, i64, p]
+        L.vitattn_test_host_plan.restype = ctypes.c_int
         L.vitattn_strerror.argtypes = [i32]
         L.vitattn_strerror.restype = ctypes.c_char_p
         for f in (L.vitattn_forward, L.vitattn_forward_checked, L.vitattn_test_forward_flags,
@@ -116,6 +118,18 @@ def version() -> int:
 
 def launches_per_call() -> int:
     return int(lib().vitattn_launches_per_call())
+
+
+def host_plan(B, H, D):
+    """How the host-buffer entry cuts [B, N, H, D] into copy/kernel groups:
+    (images per group, groups per image -- 1 when heads are not cut, else
+    part g of an image's heads is g*H//G .. (g+1)*H//G - 1 -- and groups).
+    No CUDA call (a test hook of the library)."""
+    out = (ctypes.c_int64 * 3)()
+    rc = lib().vitattn_test_host_plan(B, H, D, ctypes.cast(out, ctypes.c_void_p))
+    if rc:
+        raise VitAttnError(rc)
+    return tuple(int(x) for x in out)
 
 
 def check_args(q, k, v, out, B, N, H, D, scale, dtype) -> int:
