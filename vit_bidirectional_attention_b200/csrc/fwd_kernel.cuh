@@ -1,8 +1,11 @@
-// fwd_kernel.cuh -- sm_100a forward kernel of non-causal multi-head attention.
+// fwd_kernel.cuh -- sm_100a forward kernel of multi-head attention (no mask
+// by default; cross lengths, the aligned causal mask, grouped-query heads,
+// ragged batches and token-strided inputs are variants of the same body).
 //
-// One CTA owns one (batch b, head h) pair and up to two 128-row query tiles of
-// it (256 query rows).  K and V stream through a shared-memory ring in blocks
-// of 128 keys.  Per key block j and query tile t:
+// A work item is one (batch b, head h) pair and up to two 128-row query tiles
+// of it (256 query rows); a CTA runs one item, or loops over items.  K and V
+// stream through a shared-memory ring in blocks of 128 keys.  Per key block j
+// and query tile t:
 //
 //   S_t   = Q_t K_j^T                    tcgen05.mma, A = Q (smem), B = K (smem), f32 in TMEM
 //   P_t   = exp2(S_t * c - m_t)          softmax warpgroup t, one thread per query row,
@@ -14,7 +17,10 @@
 // with the running row maximum m_t, the row sum l_t and the rescaling of O_t
 // kept exact in the online-softmax sense: O and l are always relative to the
 // same (possibly stale) maximum, so the result is O/l at the end.  l_t sums the
-// f16 probabilities themselves, i.e. the weights the P.V product really uses.
+// f32 probabilities before their rounding to f16 (within 2^-12 relative of
+// the weights the P.V product uses).  A split item (a grid too small for two
+// tiles per CTA) gives the two softmax warpgroups the two halves of ONE query
+// tile's key blocks and merges their (m, l, O) at the end.
 // The P.V product runs in f16 for both input dtypes: f16 has three more
 // mantissa bits than bf16 for P.  For bf16 inputs V is converted to f16 in shared memory
 // after it lands (exact for |v| < 2^16 apart from f16's subnormal range,
@@ -46,7 +52,8 @@
 // then for every unit s: O_t += P_s V_j, followed by S for unit s + NS in the
 // buffer P_s has just been read from.  With NS = 3 a tile's next S is
 // computed while its softmax still works on the current block; with NS = 2
-// this is the classic two-tile ping-pong.
+// this is the classic two-tile ping-pong.  A looping CTA runs an item's
+// epilogue after handing over the next item's first block.
 //
 // Tensor memory (512 columns x 128 lanes x 32 bit):
 //   [128*b, 128*b+128)  S buffer b < NS, later P (16-bit pairs in its first 64 columns)
