@@ -95,13 +95,14 @@ def cpu_model() -> str:
     return platform.processor() or "unknown"
 
 
-def timed_launches(step, steps: int, stream, event_cls, flush=None) -> float:
+def timed_launches(step, steps: int, stream, event_cls, flush=None, per_launch=None) -> float:
     """Device milliseconds of ``steps`` launches of ``step`` on ``stream``.
 
     Without ``flush``: one event pair around the back-to-back launches.  With
     ``flush`` (a callable that writes more than the L2's capacity on the same
     stream), the flush runs before every launch and only the launches are
-    timed, each between its own pair of events; their sum is returned."""
+    timed, each between its own pair of events; their sum is returned, and
+    each launch's milliseconds are appended to ``per_launch`` if it is a list."""
     if flush is None:
         ev0, ev1 = event_cls(enable_timing=True), event_cls(enable_timing=True)
         ev0.record(stream)
@@ -117,7 +118,10 @@ def timed_launches(step, steps: int, stream, event_cls, flush=None) -> float:
         step()
         b.record(stream)
     pairs[-1][1].synchronize()
-    return sum(a.elapsed_time(b) for a, b in pairs)
+    times = [a.elapsed_time(b) for a, b in pairs]
+    if per_launch is not None:
+        per_launch.extend(times)
+    return sum(times)
 
 
 def kernel_of(workload: str) -> str:
@@ -803,8 +807,9 @@ def main():
     barrier(world)
     torch.cuda.synchronize(dev)
     sampler.mark("t_start")
+    launch_ms = []
     with torch.cuda.stream(stream):
-        ms_local = timed_launches(step, args.steps, stream, torch.cuda.Event, flush)
+        ms_local = timed_launches(step, args.steps, stream, torch.cuda.Event, flush, launch_ms)
     sampler.mark("t_stop")
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -925,6 +930,11 @@ def main():
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
+        if launch_ms:  # each launch timed on its own after the L2 flush
+            srt = sorted(launch_ms)
+            result["launch_us"] = {"median": 1e3 * srt[len(srt) // 2], "min": 1e3 * srt[0],
+                                   "note": "one event pair per launch after the flush; the ~6 us launch floor of "
+                                           "that pattern is included"}
     ranks.finish(world)
     if result is not None:
         print(json.dumps(result), flush=True)

@@ -156,8 +156,10 @@ def test_timed_launches_with_flush_times_only_the_launches(steps):
         clock.now += 40.0
         clock.log.append("flush")
 
-    ms = bench.timed_launches(step, steps, "s", fake_event_cls(clock), flush=flush)
+    per = []
+    ms = bench.timed_launches(step, steps, "s", fake_event_cls(clock), flush=flush, per_launch=per)
     assert ms == 2.0 * steps
+    assert per == [2.0] * steps
     assert clock.log == ["flush", "event", "kernel", "event"] * steps
 
 
