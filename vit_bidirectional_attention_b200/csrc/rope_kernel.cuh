@@ -78,8 +78,12 @@ __device__ __forceinline__ uint2 rotate4(uint2 x, uint2 p, float4 c, float4 s, f
 
 // Heads of one token a warp handles per loop trip: their loads are all
 // issued before any is used (several rows in flight per warp), and the
-// token's cos/sin row is loaded once for all of them.
+// token's cos/sin row is loaded once for all of them.  Without the v copy a
+// head holds two rows instead of three, so twice as many fit.
 constexpr int kRopeHeadsPerWarp = 4;
+__host__ __device__ constexpr int rope_heads_per_warp(bool copy_v) {
+    return copy_v ? kRopeHeadsPerWarp : 2 * kRopeHeadsPerWarp;
+}
 
 template <bool kBF16, bool kCopyV>
 __global__ void __launch_bounds__(kRopeThreads, 4) qkv_rope_kernel(const uint8_t* __restrict__ qkv,
@@ -89,7 +93,7 @@ __global__ void __launch_bounds__(kRopeThreads, 4) qkv_rope_kernel(const uint8_t
                                                                    uint8_t* __restrict__ k,
                                                                    uint8_t* __restrict__ v, long long T,
                                                                    int H, int D) {
-    constexpr int R = kRopeHeadsPerWarp;
+    constexpr int R = rope_heads_per_warp(kCopyV);
     const int lane = threadIdx.x & 31;
     const int groups = (H + R - 1) / R;  // head groups per token
     const long long items = T * (long long)groups;

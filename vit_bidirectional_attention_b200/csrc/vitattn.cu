@@ -554,7 +554,8 @@ int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void
     if (rc) return rc;
     rc = check_device_ptrs({qkv, cs, sn, q, k, copy_v ? v : nullptr});
     if (rc) return rc;
-    const uint64_t items = (uint64_t)T * (uint64_t)((H + vitattn::kRopeHeadsPerWarp - 1) / vitattn::kRopeHeadsPerWarp);
+    const int hpw = vitattn::rope_heads_per_warp(copy_v);
+    const uint64_t items = (uint64_t)T * (uint64_t)((H + hpw - 1) / hpw);
     const uint64_t per_block = (uint64_t)(vitattn::kRopeThreads / 32);
     const uint64_t want = (items + per_block - 1) / per_block;
     const unsigned grid = (unsigned)std::min<uint64_t>(want, (uint64_t)num_sms * 8u);
