@@ -375,9 +375,10 @@ VITATTN_API int vitattn_check_args_qk_norm_rope(const void* qkv, const float* co
  * `flash_attn_gpu`: upload the inputs, run the device entry, read the
  * output back).  Here the caller supplies the device staging buffers, so
  * the library still allocates no memory.
- *   The work is cut into up to 8 groups: runs of whole images when B >= 8,
- *   otherwise groups of heads of one image (rows of at least 1 KB of each
- *   token's heads, copied with 2-D copies; heads are independent).  Group
+ *   The work is cut into groups: up to 8 runs of whole images when B >= 8,
+ *   otherwise up to 16 groups of heads of one image each (rows of at least
+ *   512 bytes of each token's heads, copied with 2-D copies; heads are
+ *   independent).  Group
  *   c's inputs are copied in while the kernel of group c-1 runs and the
  *   output of group c-2 is copied out.  The copies run on two streams the
  *   library keeps per host thread and device (created on the first call);

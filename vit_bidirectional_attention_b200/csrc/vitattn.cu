@@ -654,18 +654,20 @@ int forward_varlen_checked(const void* q, const void* k, const void* v, void* ou
 
 // ---------------------------------------------------------------- host-buffer entry
 
-// The host-buffer entry cuts the work into up to kHostChunks groups so that
-// copies and kernels overlap: the inputs of group c+1 travel host -> device
-// while the kernel of group c runs and the output of group c-1 travels back.
-// A group is a run of whole images when the batch has at least kHostChunks
-// of them; otherwise each image is cut into groups of heads (every head of
-// a token is independent), copied as 2-D copies of the heads' columns
-// (rows of at least kMinCopyRow bytes, so the copy engines stay efficient)
-// and run through the token-strided attention with a token-strided output.
-// Two copy streams per (host thread, device) carry the two directions; the
-// kernels run on the caller's stream.
-constexpr int kHostChunks = 8;
-constexpr int64_t kMinCopyRow = 1024;
+// The host-buffer entry cuts the work into groups so that copies and kernels
+// overlap: the inputs of group c+1 travel host -> device while the kernel of
+// group c runs and the output of group c-1 travels back.  A group is a run
+// of whole images (at most kImageGroups groups: every copy call costs, so
+// more, smaller groups of images measured slower) when the batch has at
+// least kImageGroups images; otherwise each image is cut into groups of
+// heads (every head of a token is independent), at most kHostChunks groups
+// in all, copied as 2-D copies of the heads' columns (rows of at least
+// kMinCopyRow bytes) and run through the token-strided attention with a
+// token-strided output.  Two copy streams per (host thread, device) carry
+// the two directions; the kernels run on the caller's stream.
+constexpr int kHostChunks = 16;
+constexpr int kImageGroups = 8;
+constexpr int64_t kMinCopyRow = 512;
 
 struct HostPipe {
     bool ready = false;
@@ -706,7 +708,7 @@ struct HostPlan {
 HostPlan host_plan(int64_t B, int64_t H, int64_t D) {
     HostPlan pl{};
     pl.groups_per_image = 1;
-    if (B < kHostChunks && H > 1) {
+    if (B < kImageGroups && H > 1) {
         const int64_t want = (kHostChunks + B - 1) / B;              // groups per image wanted
         const int64_t min_hc = (kMinCopyRow + 2 * D - 1) / (2 * D);  // heads per copy row at least
         const int64_t g = std::min<int64_t>(std::min<int64_t>(want, H / min_hc), kHostChunks / B);
@@ -716,7 +718,7 @@ HostPlan host_plan(int64_t B, int64_t H, int64_t D) {
         pl.per_chunk = 1;
         pl.nchunks = (int)(B * pl.groups_per_image);
     } else {
-        pl.per_chunk = (B + kHostChunks - 1) / kHostChunks;
+        pl.per_chunk = (B + kImageGroups - 1) / kImageGroups;
         pl.nchunks = (int)((B + pl.per_chunk - 1) / pl.per_chunk);
     }
     return pl;
