@@ -386,6 +386,32 @@ def test_bf16_v_outside_f16_range_is_reported(cuda_device):
     assert_close(run_gpu(q, k, v_ok, 0.125, synth.BF16), oracle.attention(q, k, v_ok, 0.125, synth.BF16))
 
 
+def test_bf16_v_outside_f16_range_on_the_default_entry(cuda_device):
+    """The documented contract of the unchecked entry for a bf16 V value of
+    magnitude >= 2^16 (here 2^17): the call returns OK; the column that value
+    sits in becomes non-finite in the rows of its head (its f16 conversion
+    is inf and every row gives it a nonzero weight), and every other element
+    still matches the oracle.  The checked entry reports the same input as
+    VITATTN_ERR_RANGE (test above)."""
+    import torch
+
+    q, k, v = synth.random_qkv(1, 200, 2, 64, synth.BF16, seed=3105)
+    v = v.copy()
+    v[0, 150, 1, 7] = synth.round_to_bits(np.array([2.0 ** 17], np.float32), synth.BF16)[0]
+    tq, tk, tv = (to_dev(x, synth.BF16) for x in (q, k, v))
+    out = torch.empty_like(tq)
+    rc = vitattn.forward_ptr(tq.data_ptr(), tk.data_ptr(), tv.data_ptr(), out.data_ptr(), 1, 200, 2, 64, 0.125,
+                             synth.BF16, torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    got = from_dev(out, synth.BF16)
+    bad = ~np.isfinite(got)
+    assert bad[0, :, 1, 7].all() and bad.sum() == 200
+    ref = oracle.attention(q, k, v, 0.125, synth.BF16)
+    ok = ~bad
+    assert np.max(np.abs(got[ok] - ref[ok])) <= MAX_ABS
+
+
 def test_f16_inputs_never_report_range(cuda_device):
     q, k, v = synth.random_qkv(1, 200, 2, 64, synth.F16, seed=3104)
     v = synth.round_to_bits(synth.bits_to_float32(v, synth.F16) * np.float32(8192.0), synth.F16)
