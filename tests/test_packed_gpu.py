@@ -79,11 +79,12 @@ def test_mixed_strides(cuda_device):
     assert np.array_equal(bits_of(got), bits_of(dense))
 
 
+@pytest.mark.parametrize("H,D", [(4, 64), (19, 64), (7, 32), (5, 80)])
 @pytest.mark.parametrize("normed", [False, True])
-def test_qk_prologue_matches_the_full_prologue(cuda_device, normed):
+def test_qk_prologue_matches_the_full_prologue(cuda_device, normed, H, D):
     import torch
 
-    T, H, D = 777, 4, 64
+    T = 777
     qkv = synth.make_qkv_packed(T, H, D, synth.BF16, seed=9200, std=1.5)
     cs, sn = synth.rope_tables_2d(28, 28, D)
     cs, sn = cs[:T].copy(), sn[:T].copy()

@@ -14,13 +14,17 @@
 // projection (token stride 3*H*D), and the prologue moves a third fewer bytes.
 //
 // The pass is pure HBM traffic (read 3*T*H*D elements and the tables, write
-// 3*T*H*D elements), so the design is about coalescing: one warp per (token,
-// head), lane l holding elements 4l..4l+3 of the head's q, k and v rows
-// (8-byte accesses, consecutive lanes consecutive addresses; lanes >= D/4
-// idle).  rotate_half's partner of element d is d +- D/2, which lives in
-// lane l +- D/8 (D/2 is a multiple of 4): one warp shuffle.  Arithmetic in
-// f32 (one fma per element after the sin product), one rounding to the
-// storage dtype.
+// 3*T*H*D elements), so the design is about coalescing.  A head's row takes
+// `span` lanes (the power of two >= D/4), lane l of the span holding
+// elements 4l..4l+3 (8-byte accesses, consecutive lanes consecutive
+// addresses; lanes >= D/4 of the span idle): 32 lanes for D > 64, and for
+// D <= 64 (kPair) 16, a warp then holding two consecutive heads of a token
+// side by side, so that each load or store instruction moves 2*D*2
+// contiguous bytes (256 at D = 64) instead of leaving half the warp idle.
+// rotate_half's partner of element d is d +- D/2, which lives in lane
+// l +- D/8 of the same span (D/2 is a multiple of 4): one warp shuffle.
+// Arithmetic in f32 (one fma per element after the sin product), one
+// rounding to the storage dtype.
 #pragma once
 
 #include <cstdint>
@@ -76,7 +80,7 @@ __device__ __forceinline__ uint2 rotate4(uint2 x, uint2 p, float4 c, float4 s, f
     return r;
 }
 
-// Heads of one token a warp handles per loop trip: their loads are all
+// Rows (heads) of one token a lane handles per loop trip: their loads are all
 // issued before any is used (several rows in flight per warp), and the
 // token's cos/sin row is loaded once for all of them.  Without the v copy a
 // head holds two rows instead of three, so twice as many fit.
@@ -85,7 +89,11 @@ __host__ __device__ constexpr int rope_heads_per_warp(bool copy_v) {
     return copy_v ? kRopeHeadsPerWarp : 2 * kRopeHeadsPerWarp;
 }
 
-template <bool kBF16, bool kCopyV>
+// Heads a warp holds side by side: two (16 lanes each) when D <= 64.
+__host__ __device__ constexpr bool rope_pair(int D) { return D <= 64; }
+__host__ __device__ constexpr int rope_lane_groups(int D) { return rope_pair(D) ? 2 : 1; }
+
+template <bool kBF16, bool kCopyV, bool kPair>
 __global__ void __launch_bounds__(kRopeThreads, 4) qkv_rope_kernel(const uint8_t* __restrict__ qkv,
                                                                    const float* __restrict__ cs,
                                                                    const float* __restrict__ sn,
@@ -95,34 +103,40 @@ __global__ void __launch_bounds__(kRopeThreads, 4) qkv_rope_kernel(const uint8_t
                                                                    int H, int D) {
     constexpr int R = rope_heads_per_warp(kCopyV);
     const int lane = threadIdx.x & 31;
-    const int groups = (H + R - 1) / R;  // head groups per token
+    constexpr int span = kPair ? 16 : 32;  // lanes of one head's row
+    constexpr int G = 32 / span;           // heads side by side in the warp
+    const int grp = lane / span;           // this lane's head among them
+    const int sl = lane % span;            // this lane's place in its head's row
+    constexpr int per_trip = R * G;        // heads of a token per loop trip
+    const int groups = (H + per_trip - 1) / per_trip;  // loop trips per token
     const long long items = T * (long long)groups;
     const long long stride = (long long)gridDim.x * (kRopeThreads / 32);
     const int active_lanes = D / 4;
     const int half_lanes = D / 8;
-    const bool active = lane < active_lanes;
-    const int partner = lane < half_lanes ? lane + half_lanes : lane - half_lanes;
-    const float sign = lane < half_lanes ? -1.f : 1.f;
+    const bool active = sl < active_lanes;
+    const int partner = grp * span + (sl < half_lanes ? sl + half_lanes : sl - half_lanes);
+    const float sign = sl < half_lanes ? -1.f : 1.f;
     const size_t hd2 = (size_t)H * (size_t)D * 2u;  // bytes of one token's q (or k, v) heads
     for (long long it = (long long)blockIdx.x * (kRopeThreads / 32) + (threadIdx.x >> 5); it < items;
          it += stride) {
         const long long t = it / groups;
-        const int h0 = (int)(it - t * groups) * R;
-        const int nh = min(R, H - h0);
-        // byte offsets of this lane's 4 elements of head h0 in qkv and in the outputs
-        const size_t in0 = (size_t)t * 3u * hd2 + ((size_t)h0 * (size_t)D + 4u * (size_t)lane) * 2u;
-        const size_t out0 = (size_t)t * hd2 + ((size_t)h0 * (size_t)D + 4u * (size_t)lane) * 2u;
-        const size_t head2 = (size_t)D * 2u;
+        const int h0 = (int)(it - t * groups) * per_trip;
+        const int nh = min(per_trip, H - h0);
+        // row r of this lane is head h0 + r*G + grp; byte offsets of the lane's
+        // 4 elements of row 0 in qkv and in the outputs
+        const size_t in0 = (size_t)t * 3u * hd2 + ((size_t)(h0 + grp) * (size_t)D + 4u * (size_t)sl) * 2u;
+        const size_t out0 = (size_t)t * hd2 + ((size_t)(h0 + grp) * (size_t)D + 4u * (size_t)sl) * 2u;
+        const size_t head2 = (size_t)G * (size_t)D * 2u;  // from one row of the lane to the next
         float4 c = make_float4(0.f, 0.f, 0.f, 0.f), s = c;
         uint2 xq[R], xk[R], xv[R];
         if (active) {
-            c = ld_nc_f4(cs + (size_t)t * (size_t)D + 4u * (size_t)lane);
-            s = ld_nc_f4(sn + (size_t)t * (size_t)D + 4u * (size_t)lane);
+            c = ld_nc_f4(cs + (size_t)t * (size_t)D + 4u * (size_t)sl);
+            s = ld_nc_f4(sn + (size_t)t * (size_t)D + 4u * (size_t)sl);
         }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             xq[r] = xk[r] = xv[r] = make_uint2(0u, 0u);
-            if (active && r < nh) {
+            if (active && r * G + grp < nh) {
                 const uint8_t* src = qkv + in0 + (size_t)r * head2;
                 xq[r] = ld_nc_v2(src);
                 xk[r] = ld_nc_v2(src + hd2);
@@ -135,7 +149,7 @@ __global__ void __launch_bounds__(kRopeThreads, 4) qkv_rope_kernel(const uint8_t
                                         __shfl_sync(0xffffffffu, xq[r].y, partner));
             const uint2 pk = make_uint2(__shfl_sync(0xffffffffu, xk[r].x, partner),
                                         __shfl_sync(0xffffffffu, xk[r].y, partner));
-            if (active && r < nh) {
+            if (active && r * G + grp < nh) {
                 const size_t o = out0 + (size_t)r * head2;
                 st_v2(q + o, rotate4<kBF16>(xq[r], pq, c, s, sign));
                 st_v2(k + o, rotate4<kBF16>(xk[r], pk, c, s, sign));

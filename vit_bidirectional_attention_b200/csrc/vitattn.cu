@@ -554,7 +554,7 @@ int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void
     if (rc) return rc;
     rc = check_device_ptrs({qkv, cs, sn, q, k, copy_v ? v : nullptr});
     if (rc) return rc;
-    const int hpw = vitattn::rope_heads_per_warp(copy_v);
+    const int hpw = vitattn::rope_heads_per_warp(copy_v) * vitattn::rope_lane_groups((int)D);  // per loop trip
     const uint64_t items = (uint64_t)T * (uint64_t)((H + hpw - 1) / hpw);
     const uint64_t per_block = (uint64_t)(vitattn::kRopeThreads / 32);
     const uint64_t want = (items + per_block - 1) / per_block;
@@ -565,10 +565,16 @@ int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void
     int HH = (int)H, DD = (int)D;
     void* args[9] = {&qkv8, &cs, &sn, &q8, &k8, &v8, &TT, &HH, &DD};
     const bool bf = dtype == VITATTN_BF16;
-    const void* fn = copy_v ? (bf ? reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true, true>)
-                                  : reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false, true>))
-                            : (bf ? reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true, false>)
-                                  : reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false, false>));
+    static const void* const fns[2][2][2] = {  // [bf16][copy v][pair]
+        {{reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false, false, false>),
+          reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false, false, true>)},
+         {reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false, true, false>),
+          reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<false, true, true>)}},
+        {{reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true, false, false>),
+          reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true, false, true>)},
+         {reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true, true, false>),
+          reinterpret_cast<const void*>(vitattn::qkv_rope_kernel<true, true, true>)}}};
+    const void* fn = fns[bf ? 1 : 0][copy_v ? 1 : 0][vitattn::rope_pair((int)D) ? 1 : 0];
     cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(vitattn::kRopeThreads), args, 0, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return VITATTN_OK;
@@ -586,7 +592,8 @@ int launch_norm_rope(const void* qkv, const float* cs, const float* sn, const fl
     if (rc) return rc;
     rc = check_device_ptrs({qkv, cs, sn, qw, kw, q, k, copy_v ? v : nullptr});
     if (rc) return rc;
-    const uint64_t items = (uint64_t)T * (uint64_t)((H + vitattn::kRopeHeadsPerWarp - 1) / vitattn::kRopeHeadsPerWarp);
+    const int hpw = vitattn::kRopeHeadsPerWarp * vitattn::rope_lane_groups((int)D);  // heads per loop trip
+    const uint64_t items = (uint64_t)T * (uint64_t)((H + hpw - 1) / hpw);
     const uint64_t per_block = (uint64_t)(vitattn::kRopeThreads / 32);
     const uint64_t want = (items + per_block - 1) / per_block;
     const unsigned grid =
@@ -597,11 +604,16 @@ int launch_norm_rope(const void* qkv, const float* cs, const float* sn, const fl
     int HH = (int)H, DD = (int)D;
     void* args[12] = {&qkv8, &cs, &sn, &qw, &kw, &eps, &q8, &k8, &v8, &TT, &HH, &DD};
     const bool bf = dtype == VITATTN_BF16;
-    const void* fn =
-        copy_v ? (bf ? reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true, true>)
-                     : reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false, true>))
-               : (bf ? reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true, false>)
-                     : reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false, false>));
+    static const void* const fns[2][2][2] = {  // [bf16][copy v][pair]
+        {{reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false, false, false>),
+          reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false, false, true>)},
+         {reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false, true, false>),
+          reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<false, true, true>)}},
+        {{reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true, false, false>),
+          reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true, false, true>)},
+         {reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true, true, false>),
+          reinterpret_cast<const void*>(vitattn::qkv_norm_rope_kernel<true, true, true>)}}};
+    const void* fn = fns[bf ? 1 : 0][copy_v ? 1 : 0][vitattn::rope_pair((int)D) ? 1 : 0];
     cudaError_t e = cudaLaunchKernel(fn, dim3(grid), dim3(vitattn::kRopeThreads), args, 0, stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return VITATTN_OK;
