@@ -544,7 +544,8 @@ int launch_varlen(const void* q, const void* k, const void* v, void* out, const 
 }
 
 // The prologue: a grid-stride kernel, 8 warps per block, at most 8 blocks per SM
-// (a full SM), one warp per (token, head).
+// (a full SM); a warp takes a group of one token's heads per loop trip (two
+// heads side by side per row of the group when D <= 64).
 int launch_rope(const void* qkv, const float* cs, const float* sn, void* q, void* k, void* v, int64_t T,
                 int64_t H, int64_t D, int dtype, cudaStream_t stream, bool copy_v = true) {
     int rc = check_args_rope(qkv, cs, sn, q, k, v, T, H, D, dtype, copy_v);
