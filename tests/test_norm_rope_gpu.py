@@ -92,7 +92,7 @@ def check(qkv, cs, sn, qw, kw, eps, dtype, got, rows=None):
     (333, 16, 80, synth.BF16, 0.3, 1e-6), (257, 4, 128, synth.F16, 2.0, 0.0), (196, 16, 72, synth.F16, 1.0, 1e-6),
     (64, 5, 24, synth.BF16, 40.0, 1e-6), (77, 7, 64, synth.BF16, 0.05, 0.5),
     (50, 9, 32, synth.F16, 1.0, 1e-6), (40, 11, 48, synth.BF16, 1.3, 1e-6), (31, 17, 64, synth.BF16, 1.0, 1e-6),
-    (9, 3, 16, synth.F16, 1.0, 1e-6),
+    (9, 3, 16, synth.F16, 1.0, 1e-6), (23, 5, 40, synth.BF16, 1.0, 1e-6), (19, 6, 56, synth.F16, 0.7, 1e-6),
 ])
 def test_norm_prologue_within_bound(cuda_device, T, H, D, dtype, std, eps):
     qkv = synth.make_qkv_packed(T, H, D, dtype, seed=8500 + T + D, std=std)

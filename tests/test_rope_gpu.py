@@ -72,6 +72,7 @@ def grid_tables(T, D, w=None):
     (1, 1, 16, synth.BF16), (5, 3, 64, synth.BF16), (1000, 2, 72, synth.F16),
     (333, 16, 80, synth.BF16), (257, 4, 128, synth.F16), (196, 16, 72, synth.F16), (64, 5, 24, synth.BF16),
     (50, 9, 32, synth.F16), (40, 11, 48, synth.BF16), (31, 17, 64, synth.BF16), (9, 3, 16, synth.F16),
+    (23, 5, 40, synth.BF16), (19, 6, 56, synth.F16),
 ])
 def test_prologue_within_one_ulp(cuda_device, T, H, D, dtype):
     qkv = synth.make_qkv_packed(T, H, D, dtype, seed=8000 + T + D, std=1.7)
