@@ -148,3 +148,19 @@ def test_causal_whole_slices_against_the_oracle(cuda_device, B, H, N, D):
         check(got[b:b + 1, :, h:h + 1], o, lse_l[b:b + 1, h:h + 1], lse_o, f"causal {B}x{N}x{H}x{D} ({b},{h})")
     wide, lse_w = run_ext(q, k, v, scale, True, synth.BF16, FORCE_TWO_TILES)
     assert np.array_equal(tiny, wide) and np.array_equal(lse_l, lse_w)
+
+
+def test_batched_causal_workload_sampled_parity_at_full_size(cuda_device):
+    """The causal bench workload at full size (32 x 1024 x 16 x 64 bf16, causal,
+    LSE) in the launch the bench times (default flags: one CTA per item):
+    every row of six (b, h) slices, the first, the last and four seeded ones,
+    against the oracle, output and LSE."""
+    w = synth.WORKLOADS["batched_causal"]
+    q, k, v = synth.make_qkv(w)
+    got, lse = run_ext(q, k, v, w.scale, True, w.dtype)
+    rng = np.random.Generator(np.random.PCG64(9990))
+    picks = [(0, 0), (w.B - 1, w.H - 1)] + [(int(rng.integers(w.B)), int(rng.integers(w.H))) for _ in range(4)]
+    for b, h in picks:
+        o, lse_o = oracle.attention_ext(q[b:b + 1, :, h:h + 1], k[b:b + 1, :, h:h + 1], v[b:b + 1, :, h:h + 1],
+                                        w.scale, w.dtype, causal=True)
+        check(got[b:b + 1, :, h:h + 1], o, lse[b:b + 1, h:h + 1], lse_o, f"batched_causal ({b},{h})")

@@ -105,6 +105,39 @@ def test_qk_prologue_matches_the_full_prologue(cuda_device, normed, H, D):
     assert np.array_equal(bits_of(v), qkv[:, 2])
 
 
+@pytest.mark.parametrize("name", ["layer_batched", "layer_packed_batched"])
+def test_layer_workload_sampled_parity_at_full_size(cuda_device, name):
+    """The layer bench workloads at full size (32 images of 32 x 32 patches, 16
+    heads, D = 64, bf16, the bench's seeded projection and tables) through the
+    calls the bench times: the full prologue and the dense attention, or the
+    q/k-only prologue and the attention reading v from the projection; 1024
+    seeded token-head rows against the oracle chain."""
+    import torch
+
+    w = synth.LAYER[name]
+    pw = synth.PrologueWorkload(w.name, w.images, w.grid, w.H, w.D, w.dtype, index=w.index)
+    qkv, cs, sn = synth.make_prologue(pw)
+    B, N, H, D = w.images, w.N, w.H, w.D
+    tq = to_dev(qkv, w.dtype)
+    tc, ts = torch.from_numpy(cs).cuda(), torch.from_numpy(sn).cuda()
+    if w.packed:
+        q, k, v = vitattn.qk_rope(tq, tc, ts)
+        out = vitattn.forward_strided(q.view(B, N, H, D), k.view(B, N, H, D), v.view(B, N, H, D), scale=w.scale,
+                                      checked=True)
+    else:
+        q, k, v = vitattn.qkv_rope(tq, tc, ts)
+        out = vitattn.forward(q.view(B, N, H, D), k.view(B, N, H, D), v.view(B, N, H, D), scale=w.scale, checked=True)
+    torch.cuda.synchronize()
+    rq, rk, _ = oracle.qkv_rope(qkv, cs, sn, w.dtype)
+    oq, ok = (synth.round_to_bits(x.astype(np.float32), w.dtype) for x in (rq, rk))
+    rows = np.sort(np.random.Generator(np.random.PCG64(9310)).choice(B * N * H, 1024, replace=False))
+    got = as_f64(out, w.dtype).reshape(B * N * H, D)[rows]
+    ref = oracle.attention_rows(oq.reshape(B, N, H, D), ok.reshape(B, N, H, D),
+                                np.ascontiguousarray(qkv[:, 2]).reshape(B, N, H, D), w.scale, w.dtype, rows)
+    assert np.max(np.abs(got - ref)) <= 1e-2
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= 4e-3
+
+
 def test_packed_layer_chain_against_the_oracle(cuda_device):
     """qk_rope, then the attention reading v from the projection: the layer of
     the batched workload at 4 images, against the oracle chain."""
