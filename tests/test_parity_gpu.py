@@ -316,6 +316,41 @@ def test_host_buffer_entry_head_groups(cuda_device, B, N, H, D):
     assert_close(got, from_dev(dev, synth.BF16), "host vs device entry")
 
 
+def test_host_buffer_entry_on_the_high_res_workload(cuda_device):
+    """The end-to-end call the bench times on its default workload (2 x 16384
+    x 16 x 128 bf16 from pinned host buffers: 16 groups of two heads, 2-D
+    copies, token-strided attention): seeded output rows against the oracle,
+    and every element within the tolerance (plus one bf16 ulp) of the device
+    entry's output."""
+    import torch
+
+    w = synth.WORKLOADS["high_res"]
+    q, k, v = synth.make_qkv(w)
+    per_chunk, G, n = vitattn.host_plan(w.B, w.H, w.D)
+    assert G > 1 and n == w.B * G
+    tdt = torch_dtype(w.dtype)
+    hosts = [torch.from_numpy(x.view(np.int16).copy()).view(tdt).pin_memory() for x in (q, k, v)]
+    hout = torch.full_like(hosts[0], float("nan")).pin_memory()
+    dq, dk, dv, dout = (torch.empty(q.shape, dtype=tdt, device="cuda") for _ in range(4))
+    s = torch.cuda.current_stream()
+    rc = vitattn.forward_host_ptr(*(h.data_ptr() for h in hosts), hout.data_ptr(), dq.data_ptr(),
+                                  dk.data_ptr(), dv.data_ptr(), dout.data_ptr(), w.B, w.N, w.H,
+                                  w.D, w.scale, w.dtype, s.cuda_stream)
+    assert rc == 0, vitattn.strerror(rc)
+    s.synchronize()
+    got = synth.bits_to_float32(hout.view(torch.int16).numpy().view(np.uint16), w.dtype).astype(np.float64)
+    assert np.all(np.isfinite(got))
+    flat = got.reshape(-1, w.D)
+    idx = synth.sample_rows(w, 512, seed=w.seed + 11)
+    assert_close(flat[idx], oracle.attention_rows(q, k, v, w.scale, w.dtype, idx), "high_res host entry")
+    # the device entry runs other launches (two tiles per item, no split), so
+    # the two may round a value to neighbouring bf16 numbers: one ulp of
+    # |x| is at most |x| * 2^-7
+    dev = run_gpu(q, k, v, w.scale, w.dtype)
+    assert np.all(np.abs(got - dev) <= 1e-2 + np.abs(dev) * 2.0 ** -7)
+    assert np.linalg.norm(got - dev) / np.linalg.norm(dev) <= 4e-3
+
+
 def test_pointers_of_host_memory_are_refused(cuda_device):
     # a plain (unregistered) host pointer passed as device memory is refused
     # before anything is enqueued, instead of reaching a tensor map
